@@ -1,0 +1,175 @@
+/*
+ * kda_decode.h -- C ABI of the B200 (sm_100a) KDA layer-half decode step.
+ *
+ * One call advances a batch of sequences by one token through the
+ * linear-attention ("KDA") half of a layer:
+ *
+ *   q, k, v   = W_q x, W_k x, W_v x      FP8 E4M3 weights, fp32 128x128 block scales
+ *   beta_h    = sigmoid(W_b x)_h          bf16 weights [num_heads, hidden]
+ *   alpha     = exp(-softplus(W_a_up W_a_down x))   bf16, low rank alpha_rank
+ *   k^_h      = k_h / ||k_h||_2           (a zero k_h gives k^_h = 0)
+ *   S_h      <- (I - beta_h k^ k^T) diag(alpha_h) S_h + beta_h k^ v_h^T
+ *   o_h       = S_h^T q_h                 (read out after the update)
+ *   out       = W_o concat_h(o_h)         FP8 E4M3, fp32 128x128 block scales
+ *
+ * Sources.  The layer and its fixed-size per-sequence recurrent state, updated
+ * in place by one decode kernel, are named by the TrnRT listing ("The
+ * interesting bit": linear attention with fixed-size state), the TrnRT story
+ * ("KDA (linear attention)", one fused kernel per layer half whose working set
+ * stays on chip so that only inputs, outputs and streamed weights cross HBM)
+ * and the Kiln post ("The decode kernels, and why they are opt-in": KDA decode
+ * as one kernel updating each sequence's recurrent state in place; "How was
+ * Kiln measured": FP8 weights with 128 x 128 block scales; "Expert parallelism
+ * without an all-to-all": one scale per kernel tile).  The pages print no
+ * equations; the gated delta rule above is the decode benchmark's stated
+ * workload, read with S_h stored dk x dv (key index first).
+ *
+ * Conventions for every entry point:
+ *   - Return value: KDA_OK (0) or one of the KDA_ERR_* codes below.  No C++
+ *     exception crosses this boundary.  kda_status_string() names a code and
+ *     kda_decode_last_error() gives the handle's last detailed message.
+ *   - Every tensor pointer is DEVICE memory owned by the caller (cudaMalloc,
+ *     torch, ...) unless the name says _host.  All tensors are dense and
+ *     row-major with the shapes given; base addresses must be 16-byte aligned.
+ *   - Work is enqueued asynchronously on the handle's stream.  Errors found on
+ *     the host (null or misaligned pointers, sizes) are returned before
+ *     anything is enqueued.  A device-side bounded wait that gives up sets a
+ *     status word that the next kda_decode_step / kda_decode_sync returns as
+ *     KDA_ERR_DEVICE_TIMEOUT.
+ *   - There is no CPU fallback: without a usable sm_100 device every call
+ *     fails with KDA_ERR_NO_DEVICE or KDA_ERR_CUDA.
+ *   - A handle is not thread-safe; use one handle per stream.
+ */
+#ifndef KDA_DECODE_H_
+#define KDA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_DECODE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+/* status codes */
+#define KDA_OK 0
+#define KDA_ERR_INVALID_ARG 1       /* null / misaligned pointer, batch outside [1, max_batch], bad enum   */
+#define KDA_ERR_UNSUPPORTED_SHAPE 2 /* dimensions the kernels do not cover (see kda_decode_init)           */
+#define KDA_ERR_CUDA 3              /* a CUDA runtime call failed; kda_decode_last_error() has the text     */
+#define KDA_ERR_DEVICE_TIMEOUT 4    /* a bounded device-side wait expired; outputs of that step are invalid */
+#define KDA_ERR_NO_DEVICE 5         /* no CUDA device, or the current device is not sm_100                  */
+#define KDA_ERR_OUT_OF_MEMORY 6     /* device scratch allocation failed                                     */
+
+/* out dtypes */
+#define KDA_OUT_F32 0  /* out is fp32 [B, hidden] (default)    */
+#define KDA_OUT_BF16 1 /* out is bf16 [B, hidden], RNE rounded */
+
+/* engines (kda_config.engine) */
+#define KDA_ENGINE_AUTO 0   /* pick per shape and batch                                        */
+#define KDA_ENGINE_SIMPLE 1 /* five plain CUDA-core kernels; the correctness baseline          */
+#define KDA_ENGINE_FUSED 2  /* one persistent kernel: TMA weight stream + tcgen05 projections   */
+
+typedef struct kda_config {
+    int hidden;      /* H: model width; multiple of 128                                        */
+    int num_heads;   /* nh                                                                     */
+    int head_dk;     /* dk: key/query width per head; 64 or 128                                */
+    int head_dv;     /* dv: value width per head; 64 or 128                                    */
+    int alpha_rank;  /* r: inner width of the low-rank alpha projection; multiple of 16, <= 256 */
+    int max_batch;   /* largest batch a step may pass; 1..256; sizes the handle's scratch      */
+    int out_dtype;   /* KDA_OUT_F32 or KDA_OUT_BF16                                           */
+    int engine;      /* KDA_ENGINE_*                                                          */
+    int reserved[8]; /* must be zero                                                          */
+} kda_config;
+
+/*
+ * Layer weights (device pointers, caller-owned, read-only for the library).
+ * FP8 matrices are E4M3 ("fn": bias 7, no infinities) codes, row-major
+ * [out_features, in_features]; the dequantised weight is
+ *   W[i][j] = decode(code[i][j]) * scale[i / 128][j / 128]
+ * with scale row-major [ceil(out/128), ceil(in/128)] fp32.
+ * bf16 matrices are raw bf16 bit patterns, row-major [out, in].
+ */
+typedef struct kda_weights {
+    const uint8_t *wq;       /* [nh*dk, H]  */
+    const uint8_t *wk;       /* [nh*dk, H]  */
+    const uint8_t *wv;       /* [nh*dv, H]  */
+    const uint8_t *wo;       /* [H, nh*dv]  */
+    const float *sq;         /* [nh*dk/128, H/128]  */
+    const float *sk;         /* [nh*dk/128, H/128]  */
+    const float *sv;         /* [nh*dv/128, H/128]  */
+    const float *so;         /* [H/128, nh*dv/128]  */
+    const uint16_t *wa_down; /* bf16 [r, H]      */
+    const uint16_t *wa_up;   /* bf16 [nh*dk, r]  */
+    const uint16_t *wb;      /* bf16 [nh, H]     */
+} kda_weights;
+
+typedef struct kda_handle_s *kda_handle;
+
+/* Creates a handle on the CURRENT CUDA device.  Validates the shape
+ * (hidden % 128 == 0, dk and dv in {64, 128}, nh*dk and nh*dv multiples of
+ * 128, alpha_rank a multiple of 16 in [16, 256], 1 <= max_batch <= 256) and allocates the
+ * handle's device scratch (activations between stages, a status word) with
+ * cudaMalloc.  No weights are copied.  On failure *out_handle is set to NULL. */
+KDA_API int kda_decode_init(const kda_config *cfg, kda_handle *out_handle);
+
+/* Binds a cudaStream_t (passed as void*) for all later work; NULL = legacy default stream. */
+KDA_API int kda_decode_set_stream(kda_handle h, void *cuda_stream);
+
+/*
+ * One decode step for `batch` sequences, enqueued on the handle's stream.
+ *   x            bf16 [batch, H]                       hidden state of the new token
+ *   w            weights as above (the struct itself is read on the host during the call)
+ *   state_inout  fp32 [batch, nh, dk, dv]              recurrent state, updated in place
+ *   out          [batch, H] fp32 or bf16 (cfg.out_dtype)
+ * state_inout must not overlap x, out or the weights.  Rows >= batch of any
+ * buffer are never read or written.  Returns KDA_ERR_DEVICE_TIMEOUT if an
+ * earlier step recorded a device-side timeout (the status is then cleared).
+ */
+KDA_API int kda_decode_step(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out, int batch);
+
+/*
+ * Same step with x and out in HOST memory (pinned memory gives asynchronous
+ * copies): copies x to the handle's device staging buffer, runs the step and
+ * copies out back, all on the handle's stream, then waits for the stream.
+ * The weights and the state stay in device memory.
+ */
+KDA_API int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w, float *state_inout,
+                         void *out_host, int batch);
+
+/* Waits for the handle's stream; returns the device status of the steps since
+ * the last check (KDA_OK or KDA_ERR_DEVICE_TIMEOUT) and clears it. */
+KDA_API int kda_decode_sync(kda_handle h);
+
+/* Frees the handle's scratch.  Waits for its stream first.  NULL is accepted. */
+KDA_API int kda_decode_destroy(kda_handle h);
+
+/* Engine the handle runs for `batch` (KDA_ENGINE_SIMPLE or KDA_ENGINE_FUSED). */
+KDA_API int kda_decode_engine(kda_handle h, int batch);
+
+/* Number of kernels one kda_decode_step(batch) launches. */
+KDA_API int kda_decode_launches_per_step(kda_handle h, int batch);
+
+/* Bytes of device scratch kda_decode_init allocates for cfg (host-only query). */
+KDA_API int kda_decode_scratch_bytes(const kda_config *cfg, size_t *bytes);
+
+/* Static name of a status code ("KDA_OK", ...); never NULL. */
+KDA_API const char *kda_status_string(int status);
+
+/* Last detailed error message recorded on the handle (empty string if none); never NULL. */
+KDA_API const char *kda_decode_last_error(kda_handle h);
+
+/* KDA_DECODE_ABI_VERSION of the loaded library. */
+KDA_API int kda_decode_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_DECODE_H_ */

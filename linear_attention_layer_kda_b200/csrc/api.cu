@@ -1,0 +1,328 @@
+// api.cu -- the C ABI declared in include/kda_decode.h: handle, validation, dispatch.
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <string>
+
+#include "common.cuh"
+#include "fused.cuh"
+
+struct kda_handle_s {
+    kda_config cfg{};
+    int device = -1;
+    int num_sms = 0;
+    cudaStream_t stream = nullptr;
+    void *scratch_base = nullptr;
+    size_t scratch_bytes = 0;
+    kda::Scratch s;
+    int *status_host = nullptr;  // mapped pinned status word, readable without a sync
+    int *status = nullptr;       // its device alias; kernels record KDA_ERR_DEVICE_TIMEOUT here
+    void *x_stage = nullptr;    // device staging of x for kda_decode_step_host
+    void *out_stage = nullptr;  // device staging of out for kda_decode_step_host
+    kda::FusedState fused;
+    std::string last_error;
+};
+
+namespace {
+
+int fail(kda_handle h, int code, const std::string &msg)
+{
+    if (h) h->last_error = msg;
+    return code;
+}
+
+int cuda_fail(kda_handle h, cudaError_t e, const char *what)
+{
+    std::string m = std::string(what) + ": " + cudaGetErrorString(e);
+    (void)cudaGetLastError();
+    return fail(h, KDA_ERR_CUDA, m);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int validate_config(const kda_config *c, std::string *why)
+{
+    if (!c) { *why = "null config"; return KDA_ERR_INVALID_ARG; }
+    for (int i = 0; i < 8; ++i)
+        if (c->reserved[i] != 0) { *why = "kda_config.reserved must be zero"; return KDA_ERR_INVALID_ARG; }
+    if (c->out_dtype != KDA_OUT_F32 && c->out_dtype != KDA_OUT_BF16) { *why = "bad out_dtype"; return KDA_ERR_INVALID_ARG; }
+    if (c->engine < KDA_ENGINE_AUTO || c->engine > KDA_ENGINE_FUSED) { *why = "bad engine"; return KDA_ERR_INVALID_ARG; }
+    if (c->max_batch < 1 || c->max_batch > 256) { *why = "max_batch must be in [1, 256]"; return KDA_ERR_INVALID_ARG; }
+    if (c->hidden <= 0 || c->hidden % 128 != 0 || c->hidden > 65536) { *why = "hidden must be a positive multiple of 128 (<= 65536)"; return KDA_ERR_UNSUPPORTED_SHAPE; }
+    if (c->head_dk != 64 && c->head_dk != 128) { *why = "head_dk must be 64 or 128"; return KDA_ERR_UNSUPPORTED_SHAPE; }
+    if (c->head_dv != 64 && c->head_dv != 128) { *why = "head_dv must be 64 or 128"; return KDA_ERR_UNSUPPORTED_SHAPE; }
+    if (c->num_heads < 1 || c->num_heads > 512) { *why = "num_heads must be in [1, 512]"; return KDA_ERR_UNSUPPORTED_SHAPE; }
+    if ((c->num_heads * c->head_dk) % 128 != 0 || (c->num_heads * c->head_dv) % 128 != 0) {
+        *why = "num_heads*head_dk and num_heads*head_dv must be multiples of 128";
+        return KDA_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (c->alpha_rank < 16 || c->alpha_rank > 256 || c->alpha_rank % 16 != 0) {
+        *why = "alpha_rank must be a multiple of 16 in [16, 256]";
+        return KDA_ERR_UNSUPPORTED_SHAPE;
+    }
+    return KDA_OK;
+}
+
+// Scratch layout: the simple engine's fp32 activations, then the fused engine's area.
+size_t simple_scratch_bytes(const kda_config &c)
+{
+    const size_t B = (size_t)c.max_batch, Dk = (size_t)c.num_heads * c.head_dk, Dv = (size_t)c.num_heads * c.head_dv;
+    size_t n = 0;
+    n += align_up(B * Dk * 4, 256) * 3;            // q, k, z
+    n += align_up(B * Dv * 4, 256) * 2;            // v, o
+    n += align_up(B * (size_t)c.num_heads * 4, 256);  // bpre
+    n += align_up(B * (size_t)c.alpha_rank * 4, 256); // t
+    return n;
+}
+
+size_t staging_bytes(const kda_config &c)
+{
+    return align_up((size_t)c.max_batch * c.hidden * 2, 256) + align_up((size_t)c.max_batch * c.hidden * 4, 256);
+}
+
+kda::Dims dims_of(const kda_config &c, int B)
+{
+    return kda::Dims{B, c.hidden, c.num_heads, c.head_dk, c.head_dv, c.alpha_rank};
+}
+
+int pick_engine(kda_handle h, int batch)
+{
+    if (h->cfg.engine == KDA_ENGINE_SIMPLE) return KDA_ENGINE_SIMPLE;
+    if (kda::fused_supports(dims_of(h->cfg, batch), h->num_sms)) return KDA_ENGINE_FUSED;
+    return KDA_ENGINE_SIMPLE;
+}
+
+int check_weights(kda_handle h, const kda_weights *w)
+{
+    if (!w) return fail(h, KDA_ERR_INVALID_ARG, "null weights");
+    const void *p[11] = {w->wq, w->wk, w->wv, w->wo, w->sq, w->sk, w->sv, w->so, w->wa_down, w->wa_up, w->wb};
+    static const char *names[11] = {"wq", "wk", "wv", "wo", "sq", "sk", "sv", "so", "wa_down", "wa_up", "wb"};
+    for (int i = 0; i < 11; ++i) {
+        if (!p[i]) return fail(h, KDA_ERR_INVALID_ARG, std::string("null weight pointer ") + names[i]);
+        if (!aligned16(p[i])) return fail(h, KDA_ERR_INVALID_ARG, std::string("weight pointer not 16-byte aligned: ") + names[i]);
+    }
+    return KDA_OK;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const char *pa = static_cast<const char *>(a), *pb = static_cast<const char *>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+// Host-side checks shared by both step entry points (device pointers only).
+int check_step(kda_handle h, const void *x, const kda_weights *w, const float *state, const void *out, int batch)
+{
+    if (batch < 1 || batch > h->cfg.max_batch)
+        return fail(h, KDA_ERR_INVALID_ARG, "batch must be in [1, max_batch]");
+    if (!x || !state || !out) return fail(h, KDA_ERR_INVALID_ARG, "null x, state or out");
+    if (!aligned16(x) || !aligned16(state) || !aligned16(out))
+        return fail(h, KDA_ERR_INVALID_ARG, "x, state and out must be 16-byte aligned");
+    int rc = check_weights(h, w);
+    if (rc) return rc;
+    const kda_config &c = h->cfg;
+    const size_t nx = (size_t)batch * c.hidden * 2;
+    const size_t ns = (size_t)batch * c.num_heads * c.head_dk * c.head_dv * 4;
+    const size_t no = (size_t)batch * c.hidden * (c.out_dtype == KDA_OUT_BF16 ? 2 : 4);
+    if (overlaps(state, ns, x, nx) || overlaps(state, ns, out, no))
+        return fail(h, KDA_ERR_INVALID_ARG, "state_inout overlaps x or out");
+    return KDA_OK;
+}
+
+// Reads and clears the mapped status word (call after the stream is idle, or to peek).
+int take_device_status(kda_handle h)
+{
+    volatile int *sp = h->status_host;
+    const int st = *sp;
+    if (st == KDA_OK) return KDA_OK;
+    *sp = KDA_OK;
+    if (st == KDA_ERR_DEVICE_TIMEOUT) return fail(h, st, "a device-side bounded wait expired");
+    return fail(h, st, "device reported an error");
+}
+
+int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state, void *out, int batch)
+{
+    const kda::Dims d = dims_of(h->cfg, batch);
+    cudaError_t e;
+    if (pick_engine(h, batch) == KDA_ENGINE_FUSED)
+        e = kda::fused_step(d, *w, x, state, out, h->cfg.out_dtype, h->fused, h->status, h->num_sms, h->stream);
+    else
+        e = kda::simple_step(d, *w, x, state, out, h->cfg.out_dtype, h->s, h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_decode_abi_version(void) { return KDA_DECODE_ABI_VERSION; }
+
+const char *kda_status_string(int s)
+{
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED_SHAPE: return "KDA_ERR_UNSUPPORTED_SHAPE";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT";
+    case KDA_ERR_NO_DEVICE: return "KDA_ERR_NO_DEVICE";
+    case KDA_ERR_OUT_OF_MEMORY: return "KDA_ERR_OUT_OF_MEMORY";
+    default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+const char *kda_decode_last_error(kda_handle h) { return h ? h->last_error.c_str() : ""; }
+
+int kda_decode_scratch_bytes(const kda_config *cfg, size_t *bytes)
+{
+    std::string why;
+    int rc = validate_config(cfg, &why);
+    if (rc) return rc;
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    *bytes = simple_scratch_bytes(*cfg) + staging_bytes(*cfg) + 256 +
+             kda::fused_scratch_bytes(dims_of(*cfg, cfg->max_batch));
+    return KDA_OK;
+}
+
+int kda_decode_init(const kda_config *cfg, kda_handle *out_handle)
+{
+    if (!out_handle) return KDA_ERR_INVALID_ARG;
+    *out_handle = nullptr;
+    std::string why;
+    int rc = validate_config(cfg, &why);
+    if (rc) {
+        fprintf(stderr, "kda_decode_init: %s\n", why.c_str());
+        return rc;
+    }
+    int dev = -1, ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) { (void)cudaGetLastError(); return KDA_ERR_NO_DEVICE; }
+    if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return KDA_ERR_NO_DEVICE; }
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) { (void)cudaGetLastError(); return KDA_ERR_NO_DEVICE; }
+    if (prop.major != 10) return KDA_ERR_NO_DEVICE;  // the kernels are built for sm_100a only
+
+    kda_handle h = new (std::nothrow) kda_handle_s;
+    if (!h) return KDA_ERR_OUT_OF_MEMORY;
+    h->cfg = *cfg;
+    h->device = dev;
+    h->num_sms = prop.multiProcessorCount;
+    const size_t simple_b = simple_scratch_bytes(*cfg), stage_b = staging_bytes(*cfg);
+    const size_t fused_b = kda::fused_scratch_bytes(dims_of(*cfg, cfg->max_batch));
+    h->scratch_bytes = simple_b + stage_b + 256 + fused_b;
+    cudaError_t e = cudaMalloc(&h->scratch_base, h->scratch_bytes);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        delete h;
+        return KDA_ERR_OUT_OF_MEMORY;
+    }
+    char *p = static_cast<char *>(h->scratch_base);
+    const size_t B = (size_t)cfg->max_batch, Dk = (size_t)cfg->num_heads * cfg->head_dk;
+    const size_t Dv = (size_t)cfg->num_heads * cfg->head_dv;
+    auto take = [&](size_t n) { char *r = p; p += align_up(n, 256); return r; };
+    h->s.q = (float *)take(B * Dk * 4);
+    h->s.k = (float *)take(B * Dk * 4);
+    h->s.z = (float *)take(B * Dk * 4);
+    h->s.v = (float *)take(B * Dv * 4);
+    h->s.o = (float *)take(B * Dv * 4);
+    h->s.bpre = (float *)take(B * cfg->num_heads * 4);
+    h->s.t = (float *)take(B * cfg->alpha_rank * 4);
+    h->x_stage = take(B * cfg->hidden * 2);
+    h->out_stage = take(B * cfg->hidden * 4);
+    (void)take(256);
+    kda::fused_bind_scratch(dims_of(*cfg, cfg->max_batch), p, fused_b, &h->fused);
+    e = cudaMemset(h->scratch_base, 0, h->scratch_bytes);
+    if (e == cudaSuccess) e = cudaHostAlloc((void **)&h->status_host, 256, cudaHostAllocMapped);
+    if (e == cudaSuccess) {
+        *h->status_host = KDA_OK;
+        e = cudaHostGetDevicePointer((void **)&h->status, h->status_host, 0);
+    }
+    if (e == cudaSuccess) e = kda::fused_init(dims_of(*cfg, cfg->max_batch), &h->fused);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        if (h->status_host) cudaFreeHost(h->status_host);
+        cudaFree(h->scratch_base);
+        delete h;
+        return KDA_ERR_CUDA;
+    }
+    *out_handle = h;
+    return KDA_OK;
+}
+
+int kda_decode_set_stream(kda_handle h, void *stream)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    h->stream = static_cast<cudaStream_t>(stream);
+    return KDA_OK;
+}
+
+int kda_decode_engine(kda_handle h, int batch)
+{
+    if (!h || batch < 1 || batch > h->cfg.max_batch) return -KDA_ERR_INVALID_ARG;
+    return pick_engine(h, batch);
+}
+
+int kda_decode_launches_per_step(kda_handle h, int batch)
+{
+    if (!h || batch < 1 || batch > h->cfg.max_batch) return -KDA_ERR_INVALID_ARG;
+    if (pick_engine(h, batch) == KDA_ENGINE_FUSED) return kda::fused_launches();
+    return h->cfg.head_dk == h->cfg.head_dv ? kda::simple_launches() : kda::simple_launches() + 1;
+}
+
+int kda_decode_step(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out, int batch)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    int rc = check_step(h, x, w, state_inout, out, batch);
+    if (rc) return rc;
+    // A timeout recorded by an earlier step is reported (and cleared) here.
+    rc = take_device_status(h);
+    if (rc) return rc;
+    return enqueue_step(h, x, w, state_inout, out, batch);
+}
+
+int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w, float *state_inout,
+                         void *out_host, int batch)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    if (!x_host || !out_host) return fail(h, KDA_ERR_INVALID_ARG, "null host buffer");
+    int rc = check_step(h, h->x_stage, w, state_inout, h->out_stage, batch);
+    if (rc) return rc;
+    rc = take_device_status(h);
+    if (rc) return rc;
+    const size_t nx = (size_t)batch * h->cfg.hidden * 2;
+    const size_t no = (size_t)batch * h->cfg.hidden * (h->cfg.out_dtype == KDA_OUT_BF16 ? 2 : 4);
+    cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, nx, cudaMemcpyHostToDevice, h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "copying x to the device");
+    rc = enqueue_step(h, h->x_stage, w, state_inout, h->out_stage, batch);
+    if (rc) return rc;
+    e = cudaMemcpyAsync(out_host, h->out_stage, no, cudaMemcpyDeviceToHost, h->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "copying out to the host");
+    return take_device_status(h);
+}
+
+int kda_decode_sync(kda_handle h)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
+    return take_device_status(h);
+}
+
+int kda_decode_destroy(kda_handle h)
+{
+    if (!h) return KDA_OK;
+    int rc = KDA_OK;
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    kda::fused_destroy(&h->fused);
+    if (h->status_host && cudaFreeHost(h->status_host) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    if (cudaFree(h->scratch_base) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    delete h;
+    return rc;
+}
+
+}  // extern "C"
