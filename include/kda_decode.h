@@ -165,6 +165,17 @@ KDA_API const char *kda_status_string(int status);
 /* Last detailed error message recorded on the handle (empty string if none); never NULL. */
 KDA_API const char *kda_decode_last_error(kda_handle h);
 
+/* Intermediates of the most recent step, for stage-by-stage diagnosis (which =):      */
+#define KDA_DEBUG_Q 0        /* fp32 [batch, nh*dk]  q = W_q x                            */
+#define KDA_DEBUG_K 1        /* fp32 [batch, nh*dk]  k = W_k x (before normalisation)     */
+#define KDA_DEBUG_V 2        /* fp32 [batch, nh*dv]  v = W_v x                            */
+#define KDA_DEBUG_BETA_PRE 3 /* fp32 [batch, nh]     W_b x (before the sigmoid)           */
+#define KDA_DEBUG_T 4        /* fp32 [batch, r]      W_a_down x                           */
+
+/* Copies `bytes` of intermediate `which` of the last step into device buffer `dst`,
+ * ordered on the handle's stream (bytes must not exceed the tensor's size at max_batch). */
+KDA_API int kda_decode_debug_copy(kda_handle h, int which, void *dst, size_t bytes);
+
 /* KDA_DECODE_ABI_VERSION of the loaded library. */
 KDA_API int kda_decode_abi_version(void);
 

@@ -32,8 +32,9 @@ KDA_ENGINE_FUSED = 2
 EXPORTS = (
     "kda_decode_init", "kda_decode_set_stream", "kda_decode_step", "kda_decode_step_host", "kda_decode_sync",
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
-    "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version",
+    "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
 )
+KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
 
 
 class KdaError(RuntimeError):
@@ -86,6 +87,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_status_string": (ctypes.c_char_p, [I]),
         "kda_decode_last_error": (ctypes.c_char_p, [P]),
         "kda_decode_abi_version": (I, []),
+        "kda_decode_debug_copy": (I, [P, I, P, ctypes.c_size_t]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -140,6 +142,10 @@ def kda_decode_scratch_bytes(cfg: kda_config) -> int:
     n = ctypes.c_size_t()
     _check(load().kda_decode_scratch_bytes(ctypes.byref(cfg), ctypes.byref(n)), "kda_decode_scratch_bytes")
     return n.value
+
+
+def kda_decode_debug_copy(h: int, which: int, dst: int, nbytes: int) -> None:
+    _check(load().kda_decode_debug_copy(h, which, dst, nbytes), "kda_decode_debug_copy", h)
 
 
 def kda_status_string(status: int) -> str:
@@ -209,6 +215,17 @@ class KdaDecoder:
 
     def sync(self) -> None:
         kda_decode_sync(self.h)
+
+    def debug_tensor(self, which: int, batch: int):
+        """fp32 copy of one intermediate of the last step (KDA_DEBUG_*), shape [batch, n]."""
+        c = self.cfg
+        n = {KDA_DEBUG_Q: c.num_heads * c.head_dk, KDA_DEBUG_K: c.num_heads * c.head_dk,
+             KDA_DEBUG_V: c.num_heads * c.head_dv, KDA_DEBUG_BETA_PRE: c.num_heads,
+             KDA_DEBUG_T: c.alpha_rank}[which]
+        t = self._torch.empty(batch, n, device="cuda", dtype=self._torch.float32)
+        self._bind_stream()
+        kda_decode_debug_copy(self.h, which, t.data_ptr(), t.numel() * 4)
+        return t
 
     def engine(self, batch: int) -> int:
         return kda_decode_engine(self.h, batch)

@@ -91,7 +91,7 @@ kda::Dims dims_of(const kda_config &c, int B)
 int pick_engine(kda_handle h, int batch)
 {
     if (h->cfg.engine == KDA_ENGINE_SIMPLE) return KDA_ENGINE_SIMPLE;
-    if (kda::fused_supports(dims_of(h->cfg, batch), h->num_sms)) return KDA_ENGINE_FUSED;
+    if (h->fused.bytes && kda::fused_supports(dims_of(h->cfg, batch), h->num_sms)) return KDA_ENGINE_FUSED;
     return KDA_ENGINE_SIMPLE;
 }
 
@@ -136,10 +136,13 @@ int check_step(kda_handle h, const void *x, const kda_weights *w, const float *s
 int take_device_status(kda_handle h)
 {
     volatile int *sp = h->status_host;
-    const int st = *sp;
+    const int st = sp[0], where = sp[1];
     if (st == KDA_OK) return KDA_OK;
-    *sp = KDA_OK;
-    if (st == KDA_ERR_DEVICE_TIMEOUT) return fail(h, st, "a device-side bounded wait expired");
+    sp[0] = KDA_OK;
+    sp[1] = 0;
+    h->fused.needs_reset = true;  // flags and counters of the aborted step are inconsistent
+    if (st == KDA_ERR_DEVICE_TIMEOUT)
+        return fail(h, st, "a device-side bounded wait expired (wait site " + std::to_string(where) + ")");
     return fail(h, st, "device reported an error");
 }
 
@@ -148,7 +151,7 @@ int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state
     const kda::Dims d = dims_of(h->cfg, batch);
     cudaError_t e;
     if (pick_engine(h, batch) == KDA_ENGINE_FUSED)
-        e = kda::fused_step(d, *w, x, state, out, h->cfg.out_dtype, h->fused, h->status, h->num_sms, h->stream);
+        e = kda::fused_step(d, *w, x, state, out, h->cfg.out_dtype, h->fused, h->s, h->status, h->stream);
     else
         e = kda::simple_step(d, *w, x, state, out, h->cfg.out_dtype, h->s, h->stream);
     if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
@@ -183,8 +186,14 @@ int kda_decode_scratch_bytes(const kda_config *cfg, size_t *bytes)
     int rc = validate_config(cfg, &why);
     if (rc) return rc;
     if (!bytes) return KDA_ERR_INVALID_ARG;
+    int sms = 148, dev = 0;  // without a device, size for a 148-SM B200
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) sms = n;
+    }
+    (void)cudaGetLastError();
     *bytes = simple_scratch_bytes(*cfg) + staging_bytes(*cfg) + 256 +
-             kda::fused_scratch_bytes(dims_of(*cfg, cfg->max_batch));
+             kda::fused_scratch_bytes(dims_of(*cfg, cfg->max_batch), sms);
     return KDA_OK;
 }
 
@@ -211,7 +220,7 @@ int kda_decode_init(const kda_config *cfg, kda_handle *out_handle)
     h->device = dev;
     h->num_sms = prop.multiProcessorCount;
     const size_t simple_b = simple_scratch_bytes(*cfg), stage_b = staging_bytes(*cfg);
-    const size_t fused_b = kda::fused_scratch_bytes(dims_of(*cfg, cfg->max_batch));
+    const size_t fused_b = cfg->engine == KDA_ENGINE_SIMPLE ? 0 : kda::fused_scratch_bytes(dims_of(*cfg, cfg->max_batch), h->num_sms);
     h->scratch_bytes = simple_b + stage_b + 256 + fused_b;
     cudaError_t e = cudaMalloc(&h->scratch_base, h->scratch_bytes);
     if (e != cudaSuccess) {
@@ -233,11 +242,12 @@ int kda_decode_init(const kda_config *cfg, kda_handle *out_handle)
     h->x_stage = take(B * cfg->hidden * 2);
     h->out_stage = take(B * cfg->hidden * 4);
     (void)take(256);
-    kda::fused_bind_scratch(dims_of(*cfg, cfg->max_batch), p, fused_b, &h->fused);
+    kda::fused_bind_scratch(dims_of(*cfg, cfg->max_batch), h->num_sms, p, fused_b, &h->fused);
     e = cudaMemset(h->scratch_base, 0, h->scratch_bytes);
     if (e == cudaSuccess) e = cudaHostAlloc((void **)&h->status_host, 256, cudaHostAllocMapped);
     if (e == cudaSuccess) {
-        *h->status_host = KDA_OK;
+        h->status_host[0] = KDA_OK;
+        h->status_host[1] = 0;
         e = cudaHostGetDevicePointer((void **)&h->status, h->status_host, 0);
     }
     if (e == cudaSuccess) e = kda::fused_init(dims_of(*cfg, cfg->max_batch), &h->fused);
@@ -311,6 +321,27 @@ int kda_decode_sync(kda_handle h)
     cudaError_t e = cudaStreamSynchronize(h->stream);
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
     return take_device_status(h);
+}
+
+int kda_decode_debug_copy(kda_handle h, int which, void *dst, size_t bytes)
+{
+    if (!h || !dst) return KDA_ERR_INVALID_ARG;
+    const kda_config &c = h->cfg;
+    const size_t B = (size_t)c.max_batch;
+    const float *src = nullptr;
+    size_t n = 0;
+    switch (which) {
+    case KDA_DEBUG_Q: src = h->s.q; n = B * c.num_heads * c.head_dk; break;
+    case KDA_DEBUG_K: src = h->s.k; n = B * c.num_heads * c.head_dk; break;
+    case KDA_DEBUG_V: src = h->s.v; n = B * c.num_heads * c.head_dv; break;
+    case KDA_DEBUG_BETA_PRE: src = h->s.bpre; n = B * c.num_heads; break;
+    case KDA_DEBUG_T: src = h->s.t; n = B * c.alpha_rank; break;
+    default: return fail(h, KDA_ERR_INVALID_ARG, "unknown debug tensor");
+    }
+    if (bytes > n * 4) return fail(h, KDA_ERR_INVALID_ARG, "debug copy larger than the tensor");
+    cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "debug copy");
+    return KDA_OK;
 }
 
 int kda_decode_destroy(kda_handle h)

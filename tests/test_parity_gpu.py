@@ -150,3 +150,33 @@ def test_invalid_arguments_rejected_before_launch():
     with pytest.raises(binding.KdaError):
         binding.kda_decode_step(dec.h, x.data_ptr(), w2, st.data_ptr(), out.data_ptr(), 1)
     dec.close()
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+def test_stage_intermediates_match_oracle(engine):
+    """Block-by-block check of the projection stage: q, k, v, W_b x and W_a_down x."""
+    import oracle
+    import torch
+    from linear_attention_layer_kda_b200 import tensors
+    shape = I.CONFIGS[1]
+    inp = I.generate(shape)
+    dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, 8,
+                             engine=engine)
+    w = tensors.weights_struct(tensors.to_device_weights(inp))
+    st = tensors.state_tensor(inp.state0)
+    out = torch.empty(8, shape.hidden, device="cuda")
+    dec.step(tensors.bf16_tensor(inp.x[0]), w, st, out)
+    dec.sync()
+    m = oracle.OracleModel(inp)
+    S = inp.state0.astype(np.float64).copy()
+    _, dbg = m.step(inp.x[0], S, debug=True)
+    bpre_ref = np.log(dbg["beta"] / (1.0 - dbg["beta"]))
+    checks = [(binding.KDA_DEBUG_Q, dbg["q"]), (binding.KDA_DEBUG_K, dbg["k"]), (binding.KDA_DEBUG_V, dbg["v"]),
+              (binding.KDA_DEBUG_BETA_PRE, bpre_ref), (binding.KDA_DEBUG_T, dbg["t"])]
+    for which, ref in checks:
+        got = dec.debug_tensor(which, 8).double().cpu().numpy()
+        # per 128-row block error, reported on failure
+        err = np.abs(got - ref).max() / np.abs(ref).max()
+        blocks = [np.abs(got[:, i:i + 128] - ref[:, i:i + 128]).max() for i in range(0, ref.shape[1], 128)]
+        assert err < 1e-4, f"debug tensor {which}: max rel err {err:.3e}; per-block abs err {blocks}"
+    dec.close()
