@@ -228,7 +228,7 @@ def run_ours(args, shape, rank, world, local_rank):
     clk = ClockSampler(gpu_id_for(local_rank), os.path.join(args.outdir, f"clocks_rank{rank}.csv")) \
         if rank == 0 else None
     # untimed load window so the clock sampler sees the step loop for about a second
-    t_end = time.perf_counter() + (1.0 if clk else 0.0)
+    t_end = time.perf_counter() + (args.clock_window if clk else 0.0)
     i = 0
     while time.perf_counter() < t_end:
         one(i)
@@ -267,7 +267,7 @@ def run_ours(args, shape, rank, world, local_rank):
     if rank == 0:
         xh = torch.from_numpy(inp.x[0].view(np.int16)).view(torch.bfloat16).pin_memory()
         oh = torch.empty(B, shape.hidden, dtype=torch.float32).pin_memory()
-        n_e2e = max(10, min(args.steps, 2000))
+        n_e2e = args.e2e_steps if args.e2e_steps > 0 else max(10, min(args.steps, 2000))
         for i in range(3):
             dec.step_host(xh, ws[i % R], states[i % R], oh)
         t0 = time.perf_counter()
@@ -352,6 +352,9 @@ def main(argv=None):
     ap.add_argument("--engine", type=int, default=0, help="0 auto, 1 simple, 2 fused")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-window", type=float, default=1.0,
+                    help="seconds of untimed steps while nvidia-smi samples clocks before the timed region")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the host-buffer end-to-end loop")
     ap.add_argument("--outdir", default=os.path.join(ROOT, "gpurun_out"))
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)

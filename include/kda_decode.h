@@ -171,6 +171,8 @@ KDA_API const char *kda_decode_last_error(kda_handle h);
 #define KDA_DEBUG_V 2        /* fp32 [batch, nh*dv]  v = W_v x                            */
 #define KDA_DEBUG_BETA_PRE 3 /* fp32 [batch, nh]     W_b x (before the sigmoid)           */
 #define KDA_DEBUG_T 4        /* fp32 [batch, r]      W_a_down x                           */
+#define KDA_DEBUG_TRACE 5    /* uint64 [num_SMs][32] fused-kernel timeline stamps (ns); only in
+                                libraries built with -DKDA_TRACE, else KDA_ERR_INVALID_ARG */
 
 /* Copies `bytes` of intermediate `which` of the last step into device buffer `dst`,
  * ordered on the handle's stream (bytes must not exceed the tensor's size at max_batch). */

@@ -336,6 +336,11 @@ int kda_decode_debug_copy(kda_handle h, int which, void *dst, size_t bytes)
     case KDA_DEBUG_V: src = h->s.v; n = B * c.num_heads * c.head_dv; break;
     case KDA_DEBUG_BETA_PRE: src = h->s.bpre; n = B * c.num_heads; break;
     case KDA_DEBUG_T: src = h->s.t; n = B * c.alpha_rank; break;
+    case KDA_DEBUG_TRACE:
+        if (!h->fused.trace) return fail(h, KDA_ERR_INVALID_ARG, "library built without KDA_TRACE");
+        src = reinterpret_cast<const float *>(h->fused.trace);
+        n = (size_t)h->fused.num_ctas * kda::kTraceSlots * 2;
+        break;
     default: return fail(h, KDA_ERR_INVALID_ARG, "unknown debug tensor");
     }
     if (bytes > n * 4) return fail(h, KDA_ERR_INVALID_ARG, "debug copy larger than the tensor");

@@ -49,13 +49,39 @@ constexpr int kThreads = 512;
 constexpr int kMaxBP = 64;
 constexpr int kTileBytes = 128 * 128;
 constexpr int kHeadsPerGroup = 8;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;   // ring stages (weight tile + activation planes)
+constexpr int kMaxAcc = 8;       // TMEM accumulator buffers
+constexpr int kMaxTilesPerCta = 512;
 constexpr int kTmemCols = 512;
 
-// counters
+// Optional timeline (compile with -DKDA_TRACE): per CTA, kTraceSlots global-timer stamps.
+#ifdef KDA_TRACE
+#define KDA_TR(P, slot)                                                                       \
+    do {                                                                                      \
+        if ((P).trace) (P).trace[(size_t)blockIdx.x * kTraceSlots + (slot)] = globaltimer_ns(); \
+    } while (0)
+#else
+#define KDA_TR(P, slot) \
+    do {                \
+    } while (0)
+#endif
+enum TraceSlot {
+    TR_START = 0, TR_XREADY, TR_FIRST_MMA, TR_QKV_DONE, TR_EPI_DONE, TR_XQ_DONE, TR_GATES_DONE,
+    TR_UNIT0 = 7,  /* 3 stamps per unit: claimed, inputs ready, done; 4 units */
+    TR_O_WAIT0 = 19, TR_O_READY0, TR_O_READY_LAST, TR_END, TR_LAST_REDUCE_START, TR_LAST_REDUCE_END,
+    TR_TILE_TMA = 32, TR_TILE_MMA = 64, TR_TILE_EPI = 96, TR_TILE_TMA_RET = 128, TR_TILE_ACT = 160 /* per tile i < 32 */
+};
+
+// counters (uint32, monotonic across steps; targets are multiples of the step count)
+//   C_XQ          x K-blocks split into planes (B per K block per step)
+//   C_GATE        gate rows finished
+//   C_CLAIM0/1    state-unit claim counter of even / odd steps
+//   C_ABORT       set by any wait that gives up
+//   off_oready+kb state units done for o K-block kb (B per step)
+//   off_rb+key    segments published for row block key (q, k, v, o row blocks)
 constexpr int C_XQ = 0, C_GATE = 1, C_CLAIM0 = 2, C_ABORT = 4, C_FIXED = 16;
 
-struct VecSmem {
+struct __align__(16) VecSmem {
     float q[256], k[256], a[256];  // per head of the unit: q, k^, alpha  (heads_per_unit * dk)
     float v[128], u[128], o[128];  // per virtual column of the unit
     float t[256];                  // W_a_down x of the unit's sequence
@@ -67,24 +93,27 @@ struct VecSmem {
 struct FusedParams {
     CUtensorMap tm_w[4];  // W_q, W_k, W_v, W_o: uint8 [rows, K], box 128 x 128, 128B swizzle
     CUtensorMap tm_xq;    // x planes: [2*BP, H], box [2*BP, 128]
-    CUtensorMap tm_oq;    // o planes: [4*BP, Dv], box [4*BP, 128]
+    CUtensorMap tm_oq;    // o planes (+ scale rows when they fit in one 256-row box)
+    CUtensorMap tm_osc;   // o scale rows alone, used when 4*BP + scale rows > 256
     const float *wscale[4];
     const uint16_t *x, *wa_down, *wa_up, *wb;
     float *state;
     void *out;
-    uint8_t *xq, *oq;
-    float *xscale, *oscale, *part;
+    uint8_t *xq, *oq;  // planes + scale rows
+    float *part;
     float *q, *k, *v, *bpre, *t;
     uint32_t *ctr;
+    uint64_t *trace;  // null unless built with KDA_TRACE
     const TileEntry *tiles;
     const uint32_t *cta_off;
     int *status;
+    const uint2 *rbinfo;  // per row-block key: (first partial slot, segments)
     int B, H, nh, dk, dv, r;
-    int nKBx, nKBo, nRBq, nRBv;
-    int off_head, off_oready, off_rb, off_out;
-    uint32_t epoch, t_xq, t_gate, t_head, t_o;
+    int nKBx, nKBo, nRBq, nRBv, nRBo;
+    int off_oready, off_rb;
+    uint32_t epoch, t_xq, t_gate, t_o;
     uint64_t timeout_ns;
-    int out_bf16, stages, stage_bytes, skip_gate_release;
+    int out_bf16, stages, stage_bytes, nacc, skip_gate_release;
 };
 
 struct Ctl {
@@ -92,9 +121,15 @@ struct Ctl {
     volatile int *sh_abort;
 };
 
-__device__ __forceinline__ bool should_stop(const Ctl &c)
+// Abort check on the shared-memory flag; the global flag (set by another CTA) is read at
+// most every 20 us per waiting thread, via poll_abort.
+__device__ __forceinline__ bool should_stop(const Ctl &c) { return *c.sh_abort != 0; }
+
+__device__ __forceinline__ bool poll_abort(const Ctl &c, uint64_t now, uint64_t &next)
 {
     if (*c.sh_abort) return true;
+    if (now < next) return false;
+    next = now + 20000;
     if (*(volatile uint32_t *)(c.P.ctr + C_ABORT) != 0u) {
         *c.sh_abort = 1;
         return true;
@@ -116,11 +151,13 @@ __device__ bool wait_bar(uint64_t *b, uint32_t parity, const Ctl &c, int where)
 {
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    uint64_t next = t0 + 20000;
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(b, parity)) return true;
         if ((it & 15u) == 0u) {
-            if (should_stop(c)) return false;
-            if (globaltimer_ns() - t0 > c.P.timeout_ns) {
+            const uint64_t now = globaltimer_ns();
+            if (poll_abort(c, now, next)) return false;
+            if (now - t0 > c.P.timeout_ns) {
                 raise_abort(c, where);
                 return false;
             }
@@ -140,17 +177,45 @@ __device__ bool wait_count(const uint32_t *p, uint32_t target, const Ctl &c, int
 {
     if ((int32_t)(ld_acquire(p) - target) >= 0) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
+    uint64_t next = t0 + 20000;
+    for (;;) {
+        __nanosleep(32);
         if ((int32_t)(ld_acquire(p) - target) >= 0) return true;
-        if ((it & 15u) == 0u) {
-            if (should_stop(c)) return false;
-            if (globaltimer_ns() - t0 > c.P.timeout_ns) {
-                raise_abort(c, where);
-                return false;
-            }
+        const uint64_t now = globaltimer_ns();
+        if (poll_abort(c, now, next)) return false;
+        if (now - t0 > c.P.timeout_ns) {
+            raise_abort(c, where);
+            return false;
         }
     }
+}
+
+__device__ __forceinline__ int rb_key(const FusedParams &P, int mat, int rb)
+{
+    return mat < 2 ? mat * P.nRBq + rb : (mat == 2 ? 2 * P.nRBq + rb : 2 * P.nRBq + P.nRBv + rb);
+}
+
+// Sum of the published partials of row `r` (0..127), sequence b, of row block `key`, in slot order.
+template <int BP>
+__device__ __forceinline__ float sum_partials(const FusedParams &P, int key, int b, int r)
+{
+    const uint2 info = __ldg(P.rbinfo + key);
+    const float *base = P.part + ((size_t)info.x * BP + b) * 128 + r;
+    float s = 0.f;
+    for (uint32_t g0 = 0; g0 < info.y; g0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) v[g] = g0 + g < info.y ? __ldcg(base + (size_t)(g0 + g) * BP * 128) : 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) s += v[g];
+    }
+    return s;
+}
+
+__device__ __forceinline__ bool wait_rb(const FusedParams &P, int key, const Ctl &c, int where)
+{
+    const uint32_t nseg = __ldg(P.rbinfo + key).y;
+    return wait_count(P.ctr + P.off_rb + key, nseg * P.epoch, c, where);
 }
 
 // ---------------------------------------------------------------- activation planes
@@ -162,6 +227,15 @@ __device__ __forceinline__ float pow2_scale(float amax)
     int e;
     const float m = frexpf(amax * (1.f / 448.f), &e);
     return ldexpf(1.f, m == 0.5f ? e - 1 : e);
+}
+
+// Plane buffers hold, per K block (128 bytes of every row), NP planes of BP rows and then
+// the BP fp32 scales of the block in ceil(BP/32) extra rows ("scale rows"), so one TMA
+// copy brings a tile's activation planes and their scales.
+__host__ __device__ constexpr int scale_rows(int BP) { return (BP + 31) / 32; }
+__device__ __forceinline__ float *scale_slot(uint8_t *rowbase0, size_t pitch, int NP, int BP, int b)
+{
+    return reinterpret_cast<float *>(rowbase0 + (size_t)(NP * BP + b / 32) * pitch + (b % 32) * 4);
 }
 
 // Splits four values (already divided by their scale) into NP E4M3 planes, 4 codes per word.
@@ -203,6 +277,16 @@ __device__ __forceinline__ void st_stream_f4(float *p, float4 v)
                  : "memory");
 }
 
+// This CTA's 1/gridDim share of [p, p + bytes) -> L2 (bulk prefetch, 16-byte granules).
+__device__ __forceinline__ void prefetch_l2_slice(const void *p, size_t bytes)
+{
+    const size_t gran = (bytes / 16 + gridDim.x - 1) / gridDim.x * 16;
+    const size_t lo = (size_t)blockIdx.x * gran;
+    if (lo >= bytes) return;
+    const size_t n = (bytes - lo < gran ? bytes - lo : gran) & ~(size_t)15;
+    if (n) bulk_prefetch_l2(static_cast<const char *>(p) + lo, (uint32_t)n);
+}
+
 // ---------------------------------------------------------------- vector warps
 
 template <int BP>
@@ -221,24 +305,27 @@ __device__ void quantize_x(const FusedParams &P, int gw, int ngw, int lane)
 #pragma unroll
         for (int p = 0; p < 2; ++p)
             *reinterpret_cast<uint32_t *>(P.xq + (size_t)(p * BP + b) * P.H + kb * 128 + lane * 4) = w[p];
-        if (lane == 0) P.xscale[kb * BP + b] = s;
-        __threadfence();
+        if (lane == 0) *scale_slot(P.xq + kb * 128, P.H, 2, BP, b) = s;
         fence_proxy_async_global();
         __syncwarp();
         if (lane == 0) red_release_add(P.ctr + C_XQ, 1u);
     }
 }
 
+// Gate rows (W_b and W_a_down, bf16): one row per CTA at a time, its K range split over the
+// eight vector warps, partial sums added in warp order through shared memory.
 template <int BP>
-__device__ void gate_rows(const FusedParams &P, int gw, int ngw, int lane)
+__device__ void gate_rows(const FusedParams &P, VecSmem *vs, int vt)
 {
+    const int vw = vt >> 5, lane = vt & 31;
     const int rows = P.nh + P.r;
-    for (int it = gw; it < rows; it += ngw) {
+    const int kchunk = P.H / 8;  // multiple of 16
+    for (int it = blockIdx.x; it < rows; it += gridDim.x) {
         const uint16_t *wrow = it < P.nh ? P.wb + (size_t)it * P.H : P.wa_down + (size_t)(it - P.nh) * P.H;
         float acc[BP];
 #pragma unroll
         for (int b = 0; b < BP; ++b) acc[b] = 0.f;
-        for (int k0 = lane * 8; k0 < P.H; k0 += 256) {
+        for (int k0 = vw * kchunk + lane * 8; k0 < (vw + 1) * kchunk; k0 += 256) {
             const uint4 wr = ld_stream_v4(wrow + k0);
             const uint32_t wv[4] = {wr.x, wr.y, wr.z, wr.w};
             float wf[8];
@@ -248,37 +335,46 @@ __device__ void gate_rows(const FusedParams &P, int gw, int ngw, int lane)
                 wf[2 * j + 1] = bf16_bits_to_float(wv[j] >> 16);
             }
 #pragma unroll
-            for (int b = 0; b < BP; ++b) {
-                if (b < P.B) {
-                    const uint4 xr = __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)b * P.H + k0));
-                    const uint32_t xv[4] = {xr.x, xr.y, xr.z, xr.w};
-                    float a = acc[b];
+            for (int b0 = 0; b0 < BP; b0 += 8) {  // eight independent x loads in flight
+                uint4 xr[8];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        a = fmaf(wf[2 * j], bf16_bits_to_float(xv[j] & 0xFFFFu), a);
-                        a = fmaf(wf[2 * j + 1], bf16_bits_to_float(xv[j] >> 16), a);
+                for (int j = 0; j < 8; ++j)
+                    xr[j] = b0 + j < P.B ? __ldg(reinterpret_cast<const uint4 *>(P.x + (size_t)(b0 + j) * P.H + k0))
+                                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t xv[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
+                    float a = acc[b0 + j];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        a = fmaf(wf[2 * e], bf16_bits_to_float(xv[e] & 0xFFFFu), a);
+                        a = fmaf(wf[2 * e + 1], bf16_bits_to_float(xv[e] >> 16), a);
                     }
-                    acc[b] = a;
+                    acc[b0 + j] = a;
                 }
             }
         }
 #pragma unroll
         for (int b = 0; b < BP; ++b) {
             const float v = warp_sum(acc[b]);
-            if (lane == 0 && b < P.B) {
-                if (it < P.nh) P.bpre[(size_t)b * P.nh + it] = v;
-                else P.t[(size_t)b * P.r + (it - P.nh)] = v;
-            }
+            if (lane == 0) vs->red_w[vw][b] = v;
         }
-        __threadfence();
-        __syncwarp();
-        if (lane == 0 && !P.skip_gate_release) red_release_add(P.ctr + C_GATE, 1u);
+        named_bar(2, 256);
+        if (vt < P.B) {
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sum += vs->red_w[j][vt];
+            if (it < P.nh) P.bpre[(size_t)vt * P.nh + it] = sum;
+            else P.t[(size_t)vt * P.r + (it - P.nh)] = sum;
+        }
+        named_bar(2, 256);
+        if (vt == 0 && !P.skip_gate_release) red_release_add(P.ctr + C_GATE, 1u);
     }
 }
 
 // One state unit: sequence b, o K-block kb (heads kb*128/dv ..), all dk rows.
 template <int BP, int DK>
-__device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int b, int kb, int vt)
+__device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int b, int kb, int vt, int nu)
 {
     constexpr int RPW = DK / 8;  // rows per warp
     const int vw = vt >> 5, lane = vt & 31;
@@ -291,39 +387,66 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 #pragma unroll
     for (int r = 0; r < RPW; ++r) s[r] = ld_stream_f4(S + (size_t)(vw * RPW + r) * dv);
 
-    if (vt == 0) {
-        bool ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);
-        for (int j = 0; ok && j < hpu; ++j) ok = wait_count(P.ctr + P.off_head + h0 + j, P.t_head, c, 11);
-        vs->ok = ok;
-    }
+    // gates first: t and W_b x are final long before the unit's heads
+    if (vt == 0) vs->ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);
     named_bar(2, 256);
     if (!vs->ok) return false;
-
-    for (int i = vt; i < hpu * DK; i += 256) {
-        const size_t row = (size_t)h0 * DK + i;
-        vs->q[i] = __ldcg(P.q + (size_t)b * Dk + row);
-        vs->k[i] = __ldcg(P.k + (size_t)b * Dk + row);
-    }
-    for (int i = vt; i < 128; i += 256) vs->v[i] = __ldcg(P.v + (size_t)b * Dv + (size_t)kb * 128 + i);
     for (int j = vt; j < P.r; j += 256) vs->t[j] = __ldcg(P.t + (size_t)b * P.r + j);
     if (vt < hpu) vs->beta[vt] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + vt)));
     named_bar(2, 256);
-
     // alpha = exp(-softplus(z)) = 1 / (1 + e^z),  z = W_a_up[row] . t
     for (int i = vt; i < hpu * DK; i += 256) {
         const uint16_t *wr = P.wa_up + ((size_t)h0 * DK + i) * P.r;
         float z = 0.f;
-        for (int j = 0; j < P.r; j += 8) {
-            const uint4 w8 = __ldg(reinterpret_cast<const uint4 *>(wr + j));
-            const uint32_t wv[4] = {w8.x, w8.y, w8.z, w8.w};
+        for (int j0 = 0; j0 < P.r; j0 += 64) {
+            uint4 w8[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                z = fmaf(bf16_bits_to_float(wv[e] & 0xFFFFu), vs->t[j + 2 * e], z);
-                z = fmaf(bf16_bits_to_float(wv[e] >> 16), vs->t[j + 2 * e + 1], z);
+            for (int q8 = 0; q8 < 8; ++q8)
+                w8[q8] = j0 + q8 * 8 < P.r ? __ldg(reinterpret_cast<const uint4 *>(wr + j0 + q8 * 8)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {
+                const uint32_t wv[4] = {w8[q8].x, w8[q8].y, w8[q8].z, w8[q8].w};
+                const int j = j0 + q8 * 8;
+                if (j < P.r) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        z = fmaf(bf16_bits_to_float(wv[e] & 0xFFFFu), vs->t[j + 2 * e], z);
+                        z = fmaf(bf16_bits_to_float(wv[e] >> 16), vs->t[j + 2 * e + 1], z);
+                    }
+                }
             }
         }
         vs->a[i] = 1.f / (1.f + expf(z));
     }
+    // then the heads' q, k, v: wait for every segment of their row blocks, add the partials
+    if (vt == 0) {
+        bool ok = true;
+        const int rlo = h0 * DK / 128, rhi = ((h0 + hpu) * DK - 1) / 128;
+        for (int rb = rlo; ok && rb <= rhi; ++rb) ok = wait_rb(P, rb, c, 11) && wait_rb(P, P.nRBq + rb, c, 11);
+        if (ok) ok = wait_rb(P, 2 * P.nRBq + kb, c, 11);
+        vs->ok = ok;
+        if (nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
+    }
+    named_bar(2, 256);
+    if (!vs->ok) return false;
+    {
+        const int nqk = hpu * DK;
+        for (int it = vt; it < 2 * nqk + 128; it += 256) {
+            if (it < 2 * nqk) {
+                const int i = it % nqk, isk = it / nqk;
+                const int row = h0 * DK + i;
+                const float val = sum_partials<BP>(P, isk * P.nRBq + row / 128, b, row % 128);
+                (isk ? vs->k : vs->q)[i] = val;
+                (isk ? P.k : P.q)[(size_t)b * Dk + row] = val;  // kept for kda_decode_debug_copy
+            } else {
+                const int i = it - 2 * nqk;
+                const float val = sum_partials<BP>(P, 2 * P.nRBq + kb, b, i);
+                vs->v[i] = val;
+                P.v[(size_t)b * Dv + (size_t)kb * 128 + i] = val;
+            }
+        }
+    }
+    named_bar(2, 256);
     // ||k|| and k.q per head (one warp per head)
     if (vw < hpu) {
         float ss = 0.f, kq = 0.f;
@@ -372,16 +495,6 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         vs->o[vt] = fmaf(u, vs->kq[hx], p);
     }
     named_bar(2, 256);
-    // S' = S~ + k^ u^T, written back in place
-    const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-        const float kk = vs->k[hh * DK + vw * RPW + r];
-        float4 o;
-        o.x = fmaf(kk, u4.x, s[r].x); o.y = fmaf(kk, u4.y, s[r].y);
-        o.z = fmaf(kk, u4.z, s[r].z); o.w = fmaf(kk, u4.w, s[r].w);
-        st_stream_f4(S + (size_t)(vw * RPW + r) * dv, o);
-    }
     // o -> four E4M3 planes with one power-of-two scale for the K-block; release it
     if (vw == 0) {
         const float4 o4 = *reinterpret_cast<const float4 *>(&vs->o[vc]);
@@ -392,11 +505,20 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 #pragma unroll
         for (int p = 0; p < 4; ++p)
             *reinterpret_cast<uint32_t *>(P.oq + (size_t)(p * BP + b) * Dv + (size_t)kb * 128 + vc) = wq[p];
-        if (lane == 0) P.oscale[kb * BP + b] = sc;
-        __threadfence();
+        if (lane == 0) *scale_slot(P.oq + (size_t)kb * 128, Dv, 4, BP, b) = sc;
         fence_proxy_async_global();
         __syncwarp();
         if (lane == 0) red_release_add(P.ctr + P.off_oready + kb, 1u);
+    }
+    // S' = S~ + k^ u^T, written back in place (after the release: nothing reads it this step)
+    const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+        const float kk = vs->k[hh * DK + vw * RPW + r];
+        float4 o;
+        o.x = fmaf(kk, u4.x, s[r].x); o.y = fmaf(kk, u4.y, s[r].y);
+        o.z = fmaf(kk, u4.z, s[r].z); o.w = fmaf(kk, u4.w, s[r].w);
+        st_stream_f4(S + (size_t)(vw * RPW + r) * dv, o);
     }
     named_bar(2, 256);
     return true;
@@ -408,83 +530,144 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
     const int vt = threadIdx.x - 256, vw = vt >> 5, lane = vt & 31;
     const int gw = blockIdx.x * 8 + vw, ngw = gridDim.x * 8;
     quantize_x<BP>(P, gw, ngw, lane);
-    gate_rows<BP>(P, gw, ngw, lane);
+    if (vt == 0) KDA_TR(P, TR_XQ_DONE);
+    gate_rows<BP>(P, vs, vt);
+    if (vt == 0) KDA_TR(P, TR_GATES_DONE);
+    if (vt == 0) {
+        // warm L2 with this CTA's share of the recurrent state: units read it from L2 later
+        const size_t sbytes = (size_t)P.B * P.nh * P.dk * P.dv * 4;
+        const size_t gran = (sbytes / 16 + gridDim.x - 1) / gridDim.x * 16;
+        const size_t lo = (size_t)blockIdx.x * gran;
+        if (lo < sbytes) {
+            const size_t nb = (sbytes - lo < gran ? sbytes - lo : gran) & ~(size_t)15;
+            const uint64_t pol = policy_evict_last();
+            for (size_t o = 0; o < nb; o += 32768)
+                bulk_prefetch_l2_hint(reinterpret_cast<const char *>(P.state) + lo + o,
+                                      (uint32_t)(nb - o < 32768 ? nb - o : 32768), pol);
+        }
+    }
     const int units = P.B * P.nKBo;
     uint32_t *claim = P.ctr + C_CLAIM0 + (P.epoch & 1u);
-    for (;;) {
+    for (int nu = 0;; ++nu) {
         if (vt == 0) vs->unit = should_stop(c) ? units : (int)atomicAdd(claim, 1u);
         named_bar(2, 256);
         const int u = vs->unit;
         named_bar(2, 256);
         if (u >= units) break;
-        if (!state_unit<BP, DK>(P, vs, c, u % P.B, u / P.B, vt)) break;
+        if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu);
+        if (!state_unit<BP, DK>(P, vs, c, u % P.B, u / P.B, vt, nu)) return;
+        if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
+    }
+    // out = sum of the W_o partials: items of (row block, 32-row quarter)
+    for (int item = blockIdx.x; item < 4 * P.nRBo; item += gridDim.x) {
+        const int rb = item >> 2, key = 2 * P.nRBq + P.nRBv + rb;
+        if (vt == 0) vs->ok = wait_rb(P, key, c, 12);
+        named_bar(2, 256);
+        if (!vs->ok) return;
+        const int r = (item & 3) * 32 + lane, grow = rb * 128 + r;
+        for (int b = vw; b < P.B; b += 8) {
+            const float v = sum_partials<BP>(P, key, b, r);
+            if (P.out_bf16) static_cast<__nv_bfloat16 *>(P.out)[(size_t)b * P.H + grow] = __float2bfloat16_rn(v);
+            else static_cast<float *>(P.out)[(size_t)b * P.H + grow] = v;
+        }
+        named_bar(2, 256);
     }
 }
 
 // ---------------------------------------------------------------- projection pipeline
 
+// Shared-memory ring.  Stage s holds the weight tile (16 KB), the activation planes of the
+// same tile (up to 4 planes x BP rows x 128 bytes) and their BP scales; one producer issues
+// both copies back to back, so they sit next to each other in the TMA queue.
 struct Ring {
     uint8_t *base;
-    int stages, stage_bytes;
-    uint64_t *wfull, *afull, *wempty, *aempty, *accfull, *accempty;
-    __device__ uint8_t *w(int s) const { return base + (size_t)s * stage_bytes; }
-    __device__ uint8_t *a(int s) const { return base + (size_t)s * stage_bytes + kTileBytes; }
-    __device__ float *as(int s, int BP) const
+    int S, sbytes, NACC;
+    uint64_t *full, *empty, *accfull, *accempty;
+    __device__ uint8_t *w(int s) const { return base + (size_t)s * sbytes; }
+    __device__ uint8_t *a(int s) const { return base + (size_t)s * sbytes + kTileBytes; }
+    // scale of sequence b in the staged activation tile: row NP*BP + b/32 of a 128B-swizzled
+    // tile, 16-byte chunk ((b%32)/4) XOR (row % 8)
+    __device__ float scale(int s, int NP, int BP, int b) const
     {
-        return reinterpret_cast<float *>(base + (size_t)s * stage_bytes + kTileBytes + 4 * BP * 128);
+        const int row = NP * BP + b / 32, chunk = ((b % 32) >> 2) ^ (row & 7);
+        return *reinterpret_cast<const float *>(a(s) + row * 128 + chunk * 16 + (b & 3) * 4);
     }
 };
 
+// Warp 0, lane 0.  Weight copies run up to S tiles ahead; the activation copy of tile i is
+// issued right after its weight copy once its input is final (x split into planes, or an
+// o K-block whose state units are done).  An activation that is not ready yet is deferred
+// and polled only when no weight copy can be issued, so weights keep streaming.
 template <int BP>
-__device__ void weight_producer(const FusedParams &P, const Ring &R, const TileEntry *my, int n, const Ctl &c)
+__device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *my, int n, const Ctl &c)
 {
-    const uint64_t pol = policy_evict_first();
-    int issued = 0;
-    for (int i = 0; i < n; ++i) {
-        const TileEntry e = my[i];
-        const int s = i % R.stages;
-        const uint32_t ph = (uint32_t)(i / R.stages) & 1u;
-        if (!wait_bar(&R.wempty[s], ph ^ 1u, c, 1)) break;
-        mbar_expect_tx(&R.wfull[s], kTileBytes);
-        tma_load_2d(R.w(s), &P.tm_w[e.mat], e.kb * 128, e.rb * 128, &R.wfull[s], pol);
-        ++issued;
-    }
-    // every issued copy must land before the CTA may exit
-    for (int i = issued > R.stages ? issued - R.stages : 0; i < issued; ++i)
-        drain_bar(&R.wfull[i % R.stages], (uint32_t)(i / R.stages) & 1u, P.timeout_ns);
-}
-
-template <int BP>
-__device__ void act_producer(const FusedParams &P, const Ring &R, const TileEntry *my, int n, const Ctl &c)
-{
-    const uint64_t pol = policy_evict_last();
-    bool x_ready = false;
-    int issued = 0;
-    for (int i = 0; i < n; ++i) {
-        const TileEntry e = my[i];
-        const int s = i % R.stages;
-        const uint32_t ph = (uint32_t)(i / R.stages) & 1u;
-        if (!wait_bar(&R.aempty[s], ph ^ 1u, c, 2)) break;
+    const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
+    int nw = 0, na = 0;  // weight copies issued, activation copies issued (na <= nw)
+    bool x_ok = false;
+    uint32_t o_ok[16] = {};  // bit kb: o K-block kb known final (kb < 512)
+    uint64_t t_stall = 0, t_poll = 0, t_abort = globaltimer_ns() + 20000;
+    auto known_ready = [&](const TileEntry &e) {
+        return e.mat < 3 ? x_ok : ((o_ok[e.kb >> 5] >> (e.kb & 31)) & 1u) != 0u;
+    };
+    auto poll_ready = [&](const TileEntry &e) {
         if (e.mat < 3) {
-            if (!x_ready) {
-                if (!wait_count(P.ctr + C_XQ, P.t_xq, c, 3)) break;
-                fence_proxy_async_global();
-                x_ready = true;
-            }
-            mbar_expect_tx(&R.afull[s], 2 * BP * 128 + BP * 4);
-            tma_load_2d(R.a(s), &P.tm_xq, e.kb * 128, 0, &R.afull[s], pol);
-            bulk_load(R.as(s, BP), P.xscale + (size_t)e.kb * BP, BP * 4, &R.afull[s]);
+            if ((int32_t)(ld_acquire(P.ctr + C_XQ) - P.t_xq) < 0) return false;
+            x_ok = true;
+            KDA_TR(P, TR_XREADY);
         } else {
-            if (!wait_count(P.ctr + P.off_oready + e.kb, P.t_o, c, 4)) break;
-            fence_proxy_async_global();
-            mbar_expect_tx(&R.afull[s], 4 * BP * 128 + BP * 4);
-            tma_load_2d(R.a(s), &P.tm_oq, e.kb * 128, 0, &R.afull[s], pol);
-            bulk_load(R.as(s, BP), P.oscale + (size_t)e.kb * BP, BP * 4, &R.afull[s]);
+            if ((int32_t)(ld_acquire(P.ctr + P.off_oready + e.kb) - P.t_o) < 0) return false;
+            o_ok[e.kb >> 5] |= 1u << (e.kb & 31);
+            KDA_TR(P, TR_O_READY_LAST);
         }
-        ++issued;
+        fence_proxy_async_global();  // planes written by other SMs, read by the async proxy
+        return true;
+    };
+    while (na < n) {
+        bool progress = false;
+        while (na < nw && known_ready(my[na])) {
+            const TileEntry e = my[na];
+            const int s = na % R.S;
+            const int np = e.mat < 3 ? 2 : 4;
+            if (na < 32) KDA_TR(P, TR_TILE_ACT + na);
+            mbar_expect_tx(&R.full[s], (np * BP + scale_rows(BP)) * 128);
+            tma_load_2d(R.a(s), e.mat < 3 ? &P.tm_xq : &P.tm_oq, e.kb * 128, 0, &R.full[s], pol_a);
+            if (e.mat == 3 && 4 * BP + scale_rows(BP) > 256)
+                tma_load_2d(R.a(s) + 4 * BP * 128, &P.tm_osc, e.kb * 128, 4 * BP, &R.full[s], pol_a);
+            ++na;
+            progress = true;
+        }
+        if (nw < n && nw - na < R.S && mbar_test_wait(&R.empty[nw % R.S], ((uint32_t)(nw / R.S) & 1u) ^ 1u)) {
+            const TileEntry e = my[nw];
+            if (nw < 32) KDA_TR(P, TR_TILE_TMA + nw);
+            mbar_expect_tx(&R.full[nw % R.S], kTileBytes);
+            tma_load_2d(R.w(nw % R.S), &P.tm_w[e.mat], e.kb * 128, e.rb * 128, &R.full[nw % R.S], pol_w);
+            if (nw < 32) KDA_TR(P, TR_TILE_TMA_RET + nw);
+            ++nw;
+            t_stall = 0;
+            continue;
+        }
+        const uint64_t now = globaltimer_ns();
+        if (na < nw && now >= t_poll) {  // a poll is a global round trip: at most one per 0.5 us
+            if (poll_ready(my[na])) progress = true;
+            else t_poll = globaltimer_ns() + 500;
+        }
+        if (progress) {
+            t_stall = 0;
+            continue;
+        }
+        // nothing could be issued: give up after the timeout
+        if (poll_abort(c, now, t_abort)) break;
+        if (t_stall == 0) t_stall = now;
+        else if (now - t_stall > P.timeout_ns) {
+            raise_abort(c, 1);
+            break;
+        }
     }
-    for (int i = issued > R.stages ? issued - R.stages : 0; i < issued; ++i)
-        drain_bar(&R.afull[i % R.stages], (uint32_t)(i / R.stages) & 1u, P.timeout_ns);
+    // Every issued copy must land before the CTA may exit.  Stages whose activation copy was
+    // never issued get the missing arrival, so their phase completes when the weight lands.
+    for (int i = na; i < nw; ++i) mbar_arrive(&R.full[i % R.S]);
+    for (int i = nw > R.S ? nw - R.S : 0; i < nw; ++i)
+        drain_bar(&R.full[i % R.S], (uint32_t)(i / R.S) & 1u, P.timeout_ns);
 }
 
 template <int BP>
@@ -494,33 +677,39 @@ __device__ void mma_issuer(const FusedParams &P, const Ring &R, const TileEntry 
     int issued = 0;
     for (int i = 0; i < n; ++i) {
         const TileEntry e = my[i];
-        const int s = i % R.stages, buf = i & 1;
-        const uint32_t ph = (uint32_t)(i / R.stages) & 1u, bph = (uint32_t)(i >> 1) & 1u;
-        if (!wait_bar(&R.wfull[s], ph, c, 5)) break;
-        if (!wait_bar(&R.afull[s], ph, c, 6)) break;
+        const int s = i % R.S, buf = i % R.NACC;
+        const uint32_t ph = (uint32_t)(i / R.S) & 1u, bph = (uint32_t)(i / R.NACC) & 1u;
+        if (!wait_bar(&R.full[s], ph, c, 5)) break;
         if (!wait_bar(&R.accempty[buf], bph ^ 1u, c, 7)) break;
         tc_fence_after();
         const uint32_t idesc = e.mat < 3 ? idesc_e4m3_f32(128, 2 * BP) : idesc_e4m3_f32(128, 4 * BP);
         const uint32_t aa = smem_u32(R.w(s)), ba = smem_u32(R.a(s));
-        const uint32_t d = tmem + (uint32_t)buf * 256u;
+        const uint32_t d = tmem + (uint32_t)(buf * 4 * BP);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             mma_f8f6f4(d, sdesc_k128_sw128(aa + ks * 32), sdesc_k128_sw128(ba + ks * 32), idesc, ks > 0 ? 1u : 0u);
-        mma_commit(&R.wempty[s]);
-        mma_commit(&R.aempty[s]);
+        mma_commit(&R.empty[s]);
         mma_commit(&R.accfull[buf]);
+        if (issued == 0) KDA_TR(P, TR_FIRST_MMA);
+        if (i < 32) KDA_TR(P, TR_TILE_MMA + i);
         ++issued;
     }
     if (issued > 0) {  // the last MMAs must finish before TMEM is freed
         const int i = issued - 1;
-        drain_bar(&R.accfull[i & 1], (uint32_t)(i >> 1) & 1u, P.timeout_ns);
+        drain_bar(&R.accfull[i % R.NACC], (uint32_t)(i / R.NACC) & 1u, P.timeout_ns);
     }
 }
 
 template <int NPL, int BP>
-__device__ __forceinline__ void accumulate_tile(uint32_t taddr, const float *as, float ws, float (&acc)[BP])
+__device__ __forceinline__ void accumulate_tile(uint32_t taddr, const Ring &R, int s, float ws, float (&acc)[BP])
 {
     constexpr int N = NPL * BP;
+    constexpr bool kCache = BP <= 32;  // keep the BP combined scales in registers
+    float as[kCache ? BP : 1];
+    if (kCache) {
+#pragma unroll
+        for (int b = 0; b < (kCache ? BP : 1); ++b) as[b] = ws * R.scale(s, NPL, BP, b);
+    }
 #pragma unroll
     for (int c0 = 0; c0 < N; c0 += 16) {
         float v[16];
@@ -529,7 +718,8 @@ __device__ __forceinline__ void accumulate_tile(uint32_t taddr, const float *as,
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int b = (c0 + j) % BP;
-            acc[b] = fmaf(ws * as[b], v[j], acc[b]);
+            const float f = kCache ? as[kCache ? b : 0] : ws * R.scale(s, NPL, BP, b);
+            acc[b] = fmaf(f, v[j], acc[b]);
         }
     }
 }
@@ -542,11 +732,14 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t *b, uint32_t parity, cons
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// Warps 4-7.  After an abort the loop keeps running with the work skipped, so that all
-// 128 threads pass the same named barriers.
+// Warps 4-7: per tile, read the fp32 accumulator from TMEM, scale it and add it to the
+// running segment sum in registers; at a segment end publish the partial and release it.
+// Nothing here waits on global memory, so the MMA (up to NACC buffers ahead) never idles
+// behind a publication.  After an abort the loop keeps running with the work skipped, so
+// that all 128 threads pass the same named barriers.
 template <int BP>
 __device__ void epilogue_role(const FusedParams &P, const Ring &R, const TileEntry *my, int n, uint32_t tmem,
-                              volatile int *sh_last, const Ctl &c)
+                              const Ctl &c)
 {
     const int et = threadIdx.x - 128;  // 0..127
     const int quarter = (threadIdx.x >> 5) & 3;
@@ -557,76 +750,41 @@ __device__ void epilogue_role(const FusedParams &P, const Ring &R, const TileEnt
     float acc[BP];
 #pragma unroll
     for (int b = 0; b < BP; ++b) acc[b] = 0.f;
+    auto wscale_of = [&](const TileEntry &t) {
+        return __ldg(P.wscale[t.mat] + (size_t)t.rb * (t.mat < 3 ? P.nKBx : P.nKBo) + t.kb);
+    };
+    float ws_next = n > 0 ? wscale_of(my[0]) : 0.f;
     for (int i = 0; i < n; ++i) {
         const TileEntry e = my[i];
-        const int s = i % R.stages, buf = i & 1;
-        const uint32_t bph = (uint32_t)(i >> 1) & 1u;
-        const int nkb = e.mat < 3 ? P.nKBx : P.nKBo;
-        const float ws = __ldg(P.wscale[e.mat] + (size_t)e.rb * nkb + e.kb);
+        const int s = i % R.S, buf = i % R.NACC;
+        const uint32_t bph = (uint32_t)(i / R.NACC) & 1u;
+        const float ws = ws_next;
+        if (i + 1 < n) ws_next = wscale_of(my[i + 1]);  // one tile ahead
         if (e.flags & kSegStart) {
 #pragma unroll
             for (int b = 0; b < BP; ++b) acc[b] = 0.f;
         }
+        if (et == 0 && e.mat == 3 && (i == 0 || my[i - 1].mat != 3)) KDA_TR(P, TR_QKV_DONE);
         if (!dead && !warp_wait_bar(&R.accfull[buf], bph, c, 8)) dead = true;
         if (!dead) {
             tc_fence_after();
-            const float *as = R.as(s, BP);
-            const uint32_t taddr = taddr_base + (uint32_t)buf * 256u;
-            if (e.mat < 3) accumulate_tile<2, BP>(taddr, as, ws, acc);
-            else accumulate_tile<4, BP>(taddr, as, ws, acc);
-            mbar_arrive(&R.aempty[s]);
+            const uint32_t taddr = taddr_base + (uint32_t)(buf * 4 * BP);
+            if (e.mat < 3) accumulate_tile<2, BP>(taddr, R, s, ws, acc);
+            else accumulate_tile<4, BP>(taddr, R, s, ws, acc);
+            mbar_arrive(&R.empty[s]);  // the stage's scales are read
             tc_fence_before();
             mbar_arrive(&R.accempty[buf]);
+            if (et == 0 && i < 32) KDA_TR(P, TR_TILE_EPI + i);
         }
         if (!(e.flags & kSegEnd)) continue;
-
-        // segment done: publish the partial; the last contributor of the row block sums them
         if (!dead) {
             float *part = P.part + (size_t)e.seg * BP * 128;
 #pragma unroll
             for (int b = 0; b < BP; ++b)
                 if (b < P.B) part[b * 128 + row] = acc[b];
         }
-        __threadfence();
-        named_bar(1, 128);
-        if (et == 0) {
-            int last = 0;
-            if (!dead && !should_stop(c)) {
-                uint32_t *cnt = e.mat < 3 ? P.ctr + P.off_rb + (e.mat < 2 ? e.mat * P.nRBq : 2 * P.nRBq) + e.rb
-                                          : P.ctr + P.off_out + e.rb;
-                const uint32_t old = atom_acq_rel_add(cnt, 1u);
-                last = (old + 1u == (uint32_t)e.nseg * P.epoch) ? 1 : 0;
-            }
-            *sh_last = last;
-        }
-        named_bar(1, 128);
-        const bool last = *sh_last != 0;
-        named_bar(1, 128);
-        if (last) {
-            __threadfence();
-            const int grow = e.rb * 128 + row;
-            for (int b = 0; b < P.B; ++b) {
-                float sum = 0.f;
-                for (int g = 0; g < e.nseg; ++g)
-                    sum += __ldcg(P.part + ((size_t)(e.seg0 + g) * BP + b) * 128 + row);
-                if (e.mat == 3) {
-                    if (P.out_bf16) static_cast<__nv_bfloat16 *>(P.out)[(size_t)b * P.H + grow] = __float2bfloat16_rn(sum);
-                    else static_cast<float *>(P.out)[(size_t)b * P.H + grow] = sum;
-                } else if (e.mat == 2) {
-                    P.v[(size_t)b * P.nh * P.dv + grow] = sum;
-                } else {
-                    (e.mat == 0 ? P.q : P.k)[(size_t)b * P.nh * P.dk + grow] = sum;
-                }
-            }
-            if (e.mat < 3) {
-                __threadfence();
-                named_bar(1, 128);
-                if (et == 0) {
-                    const int hd = e.mat == 2 ? P.dv : P.dk;
-                    for (int h = e.rb * 128 / hd; h < (e.rb + 1) * 128 / hd; ++h) red_release_add(P.ctr + P.off_head + h, 1u);
-                }
-            }
-        }
+        named_bar(1, 128);  // all 128 partial rows are stored before the release
+        if (et == 0 && !dead && !*c.sh_abort) red_release_add(P.ctr + P.off_rb + rb_key(P, e.mat, e.rb), 1u);
     }
 }
 
@@ -636,42 +794,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Ring R;
+    R.S = P.stages;
+    R.sbytes = P.stage_bytes;
+    R.NACC = P.nacc;
     R.base = smem;
-    R.stages = P.stages;
-    R.stage_bytes = P.stage_bytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)P.stages * P.stage_bytes);
-    R.wfull = bars;
-    R.afull = bars + kMaxStages;
-    R.wempty = bars + 2 * kMaxStages;
-    R.aempty = bars + 3 * kMaxStages;
-    R.accfull = bars + 4 * kMaxStages;
-    R.accempty = bars + 4 * kMaxStages + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * kMaxStages + 4);
+    R.full = bars;
+    R.empty = bars + kMaxStages;
+    R.accfull = bars + 2 * kMaxStages;
+    R.accempty = bars + 2 * kMaxStages + kMaxAcc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kMaxStages + 2 * kMaxAcc);
     volatile int *sh_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *sh_last = reinterpret_cast<volatile int *>(tmem_slot + 2);
-    VecSmem *vs = reinterpret_cast<VecSmem *>(bars + 4 * kMaxStages + 8);
+    VecSmem *vs = reinterpret_cast<VecSmem *>(bars + 2 * kMaxStages + 2 * kMaxAcc + 2);
+    TileEntry *stiles = reinterpret_cast<TileEntry *>(reinterpret_cast<uint8_t *>(vs) + sizeof(VecSmem));
+
+    // this CTA's tile list -> shared memory (read by every role, once per tile)
+    const uint32_t t_begin = P.cta_off[blockIdx.x];
+    const int n = (int)(P.cta_off[blockIdx.x + 1] - t_begin);
+    for (int i = threadIdx.x; i < n; i += kThreads) stiles[i] = P.tiles[t_begin + i];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < P.stages; ++s) {
-            mbar_init(&R.wfull[s], 1);
-            mbar_init(&R.afull[s], 1);
-            mbar_init(&R.wempty[s], 1);
-            mbar_init(&R.aempty[s], 1 + 128);
+            mbar_init(&R.full[s], 2);          // weight copy + activation copy
+            mbar_init(&R.empty[s], 1 + 128);   // MMA commit + the epilogue's 128 threads
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < P.nacc; ++b) {
             mbar_init(&R.accfull[b], 1);
             mbar_init(&R.accempty[b], 128);
         }
         *sh_abort = 0;
-        *sh_last = 0;
         mbar_fence_init();
         if (blockIdx.x == 0) P.ctr[C_CLAIM0 + ((P.epoch + 1u) & 1u)] = 0u;  // next step's unit counter
+    }
+    if (warp == 3 && lane == 0) {
+        // small inputs every CTA reads soon: pull them into L2 before the weight stream queues up
+        prefetch_l2_slice(P.x, (size_t)P.B * P.H * 2);
+        prefetch_l2_slice(P.wb, (size_t)P.nh * P.H * 2);
+        prefetch_l2_slice(P.wa_down, (size_t)P.r * P.H * 2);
+        prefetch_l2_slice(P.wa_up, (size_t)P.nh * P.dk * P.r * 2);
     }
     if (warp == 0 && lane == 0) {
         for (int m = 0; m < 4; ++m) prefetch_tmap(&P.tm_w[m]);
         prefetch_tmap(&P.tm_xq);
         prefetch_tmap(&P.tm_oq);
+        if (4 * BP + scale_rows(BP) > 256) prefetch_tmap(&P.tm_osc);
     }
     if (warp == 2) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -680,19 +847,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0) KDA_TR(P, TR_START);
     const uint32_t tmem = *tmem_slot;
     const Ctl c{P, sh_abort};
-    const TileEntry *my = P.tiles + P.cta_off[blockIdx.x];
-    const int n = (int)(P.cta_off[blockIdx.x + 1] - P.cta_off[blockIdx.x]);
+    const TileEntry *my = stiles;
 
     if (warp == 0) {
-        if (lane == 0) weight_producer<BP>(P, R, my, n, c);
-    } else if (warp == 1) {
-        if (lane == 0) act_producer<BP>(P, R, my, n, c);
+        if (lane == 0) producer<BP>(P, R, my, n, c);
     } else if (warp == 2) {
         if (lane == 0) mma_issuer<BP>(P, R, my, n, tmem, c);
     } else if (warp >= 4 && warp < 8) {
-        epilogue_role<BP>(P, R, my, n, tmem, sh_last, c);
+        epilogue_role<BP>(P, R, my, n, tmem, c);
+        if (threadIdx.x == 128) KDA_TR(P, TR_EPI_DONE);
     } else if (warp >= 8) {
         vector_role<BP, DK>(P, vs, c);
     }
@@ -703,6 +869,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0) KDA_TR(P, TR_END);
 }
 
 // ---------------------------------------------------------------- host side
@@ -750,11 +917,12 @@ int bp_for(int B)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-size_t stage_bytes_for(int BP) { return align_up((size_t)kTileBytes + 4 * BP * 128 + 256, 1024); }
+// ring stage: weight tile, then up to four activation planes of BP rows and the scale rows
+size_t stage_bytes_for(int BP) { return align_up((size_t)kTileBytes + (4 * BP + scale_rows(BP)) * 128, 1024); }
 
 size_t ctr_words(const Dims &d)
 {
-    return C_FIXED + (size_t)d.nh + d.Dv() / 128 + 2 * (d.Dk() / 128) + d.Dv() / 128 + d.H / 128 + 16;
+    return C_FIXED + (size_t)d.Dv() / 128 + 2 * (d.Dk() / 128) + d.Dv() / 128 + d.H / 128 + 16;
 }
 
 template <int BP, int DK>
@@ -783,7 +951,7 @@ void *pick_kernel(int BP, int DK)
 // segment is a CTA's run inside one row block; its partial-sum slot is numbered row block
 // by row block so the segments of a row block are adjacent.
 void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, std::vector<uint32_t> *off,
-                          size_t *nseg_total)
+                          size_t *nseg_total, std::vector<uint32_t> *rbinfo)
 {
     const int nKBx = d.H / 128, nKBo = d.Dv() / 128, nRBq = d.Dk() / 128, nRBv = d.Dv() / 128, nRBo = d.H / 128;
     const int hpu = std::max(128 / d.dk, 128 / d.dv);
@@ -863,7 +1031,13 @@ void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, s
     }
     (*off)[P] = (uint32_t)tiles->size();
     *nseg_total = total;
-    (void)nRBo;
+    if (rbinfo) {
+        rbinfo->resize(2 * (size_t)nkeys);
+        for (int k = 0; k < nkeys; ++k) {
+            (*rbinfo)[2 * k] = seg0[k];
+            (*rbinfo)[2 * k + 1] = nseg[k];
+        }
+    }
     (void)nKBo;
 }
 
@@ -886,16 +1060,17 @@ size_t fused_scratch_bytes(const Dims &dmax, int num_sms)
     std::vector<TileEntry> t;
     std::vector<uint32_t> o;
     size_t nseg = 0;
-    fused_build_schedule(dmax, num_ctas_for(num_sms), &t, &o, &nseg);
+    fused_build_schedule(dmax, num_ctas_for(num_sms), &t, &o, &nseg, nullptr);
+    for (size_t c = 0; c + 1 < o.size(); ++c)
+        if (o[c + 1] - o[c] > (uint32_t)kMaxTilesPerCta) return 0;  // too many tiles per CTA: simple engine
     size_t n = 0;
-    n += align_up((size_t)2 * bpm * dmax.H, 1024);                       // x planes
-    n += align_up((size_t)(dmax.H / 128) * bpm * 4, 256);                // x scales
-    n += align_up((size_t)4 * bpm * dmax.Dv(), 1024);                     // o planes
-    n += align_up((size_t)(dmax.Dv() / 128) * bpm * 4, 256);             // o scales
+    n += align_up((size_t)(2 * bpm + scale_rows(bpm)) * dmax.H, 1024);    // x planes + scale rows
+    n += align_up((size_t)(4 * bpm + scale_rows(bpm)) * dmax.Dv(), 1024);  // o planes + scale rows
     n += align_up(nseg * bpm * 128 * 4, 256);                             // partial sums
     n += align_up(ctr_words(dmax) * 4, 256);                              // counters
     n += align_up(t.size() * sizeof(TileEntry), 256);                     // tile lists
     n += align_up(o.size() * 4, 256);
+    n += align_up((size_t)2 * (2 * (dmax.Dk() / 128) + 2 * (dmax.Dv() / 128) + dmax.H / 128) * 4, 256);  // rbinfo
     return n + 1024;
 }
 
@@ -907,23 +1082,23 @@ void fused_bind_scratch(const Dims &dmax, int num_sms, void *base, size_t bytes,
     const int bpm = bp_for(std::min(dmax.B, kMaxBP));
     fs->bp_max = bpm;
     fs->num_ctas = num_ctas_for(num_sms);
-    fused_build_schedule(dmax, fs->num_ctas, &fs->h_tiles, &fs->h_off, &fs->nseg_total);
+    fused_build_schedule(dmax, fs->num_ctas, &fs->h_tiles, &fs->h_off, &fs->nseg_total, &fs->h_rbinfo);
     fs->ntiles = fs->h_tiles.size();
+    fs->max_tiles_per_cta = 0;
+    for (int c = 0; c < fs->num_ctas; ++c)
+        fs->max_tiles_per_cta = std::max(fs->max_tiles_per_cta, (int)(fs->h_off[c + 1] - fs->h_off[c]));
     char *p = reinterpret_cast<char *>(align_up(reinterpret_cast<uintptr_t>(base), 1024));
     auto take = [&](size_t n, size_t a) { char *r = p; p += align_up(n, a); return r; };
-    fs->xq = (uint8_t *)take((size_t)2 * bpm * dmax.H, 1024);
-    fs->xscale = (float *)take((size_t)(dmax.H / 128) * bpm * 4, 256);
-    fs->oq = (uint8_t *)take((size_t)4 * bpm * dmax.Dv(), 1024);
-    fs->oscale = (float *)take((size_t)(dmax.Dv() / 128) * bpm * 4, 256);
+    fs->xq = (uint8_t *)take((size_t)(2 * bpm + scale_rows(bpm)) * dmax.H, 1024);
+    fs->oq = (uint8_t *)take((size_t)(4 * bpm + scale_rows(bpm)) * dmax.Dv(), 1024);
     fs->part = (float *)take(fs->nseg_total * bpm * 128 * 4, 256);
     fs->ctr_bytes = ctr_words(dmax) * 4;
     fs->ctr = (uint32_t *)take(fs->ctr_bytes, 256);
     fs->tiles = (TileEntry *)take(fs->h_tiles.size() * sizeof(TileEntry), 256);
     fs->cta_off = (uint32_t *)take(fs->h_off.size() * 4, 256);
-    fs->off_head = C_FIXED;
-    fs->off_oready = fs->off_head + dmax.nh;
+    fs->rbinfo = (uint32_t *)take(fs->h_rbinfo.size() * 4, 256);
+    fs->off_oready = C_FIXED;
     fs->off_rb = fs->off_oready + dmax.Dv() / 128;
-    fs->off_out = fs->off_rb + 2 * (dmax.Dk() / 128) + dmax.Dv() / 128;
 }
 
 cudaError_t fused_init(const Dims &, FusedState *fs)
@@ -934,15 +1109,26 @@ cudaError_t fused_init(const Dims &, FusedState *fs)
         if (ms > 0) fs->timeout_ns = (uint64_t)(ms * 1e6);
     }
     if (const char *e = getenv("KDA_DEBUG_SKIP_GATE_RELEASE")) fs->debug_skip_gate_release = atoi(e) != 0;
+    if (const char *e = getenv("KDA_STAGES")) fs->stages_override = atoi(e);
     cudaError_t err = cudaMemcpy(fs->tiles, fs->h_tiles.data(), fs->h_tiles.size() * sizeof(TileEntry),
                                  cudaMemcpyHostToDevice);
     if (err == cudaSuccess)
         err = cudaMemcpy(fs->cta_off, fs->h_off.data(), fs->h_off.size() * 4, cudaMemcpyHostToDevice);
+    if (err == cudaSuccess)
+        err = cudaMemcpy(fs->rbinfo, fs->h_rbinfo.data(), fs->h_rbinfo.size() * 4, cudaMemcpyHostToDevice);
+#ifdef KDA_TRACE
+    if (err == cudaSuccess) err = cudaMalloc(&fs->trace, (size_t)fs->num_ctas * kTraceSlots * 8);
+    if (err == cudaSuccess) err = cudaMemset(fs->trace, 0, (size_t)fs->num_ctas * kTraceSlots * 8);
+#endif
     fs->uploaded = err == cudaSuccess;
     return err;
 }
 
-void fused_destroy(FusedState *) {}
+void fused_destroy(FusedState *fs)
+{
+    if (fs->trace) cudaFree(fs->trace);
+    fs->trace = nullptr;
+}
 
 int fused_launches() { return 1; }
 
@@ -981,8 +1167,14 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
         for (int m = 0; m < 4; ++m) fs.map_keys[slot][m] = keys[m];
     }
     for (int m = 0; m < 4; ++m) P.tm_w[m] = fs.wmaps[slot][m];
-    if (!encode_u8_map(&P.tm_xq, fs.xq, 2 * BP, d.H, 2 * BP)) return cudaErrorInvalidValue;
-    if (!encode_u8_map(&P.tm_oq, fs.oq, 4 * BP, d.Dv(), 4 * BP)) return cudaErrorInvalidValue;
+    const int sr = scale_rows(BP);
+    if (!encode_u8_map(&P.tm_xq, fs.xq, 2 * BP + sr, d.H, 2 * BP + sr)) return cudaErrorInvalidValue;
+    if (4 * BP + sr <= 256) {
+        if (!encode_u8_map(&P.tm_oq, fs.oq, 4 * BP + sr, d.Dv(), 4 * BP + sr)) return cudaErrorInvalidValue;
+    } else {
+        if (!encode_u8_map(&P.tm_oq, fs.oq, 4 * BP + sr, d.Dv(), 4 * BP)) return cudaErrorInvalidValue;
+        if (!encode_u8_map(&P.tm_osc, fs.oq, 4 * BP + sr, d.Dv(), sr)) return cudaErrorInvalidValue;
+    }
     P.wscale[0] = w.sq;
     P.wscale[1] = w.sk;
     P.wscale[2] = w.sv;
@@ -995,8 +1187,6 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.out = out;
     P.xq = fs.xq;
     P.oq = fs.oq;
-    P.xscale = fs.xscale;
-    P.oscale = fs.oscale;
     P.part = fs.part;
     P.q = s.q;
     P.k = s.k;
@@ -1004,6 +1194,7 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.bpre = s.bpre;
     P.t = s.t;
     P.ctr = fs.ctr;
+    P.trace = fs.trace;
     P.tiles = fs.tiles;
     P.cta_off = fs.cta_off;
     P.status = status;
@@ -1017,27 +1208,29 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.nKBo = d.Dv() / 128;
     P.nRBq = d.Dk() / 128;
     P.nRBv = d.Dv() / 128;
-    P.off_head = fs.off_head;
     P.off_oready = fs.off_oready;
     P.off_rb = fs.off_rb;
-    P.off_out = fs.off_out;
+    P.rbinfo = reinterpret_cast<const uint2 *>(fs.rbinfo);
+    P.nRBo = d.H / 128;
     const uint32_t epoch = fs.epoch + 1;
     P.epoch = epoch;
     P.t_xq = (fs.cum_b + (uint32_t)d.B) * (uint32_t)P.nKBx;
     P.t_gate = epoch * (uint32_t)(d.nh + d.r);
-    P.t_head = epoch * 3u;
     P.t_o = fs.cum_b + (uint32_t)d.B;
     P.timeout_ns = fs.timeout_ns;
     P.out_bf16 = out_dtype == KDA_OUT_BF16;
     P.skip_gate_release = fs.debug_skip_gate_release;
-    const size_t sb = stage_bytes_for(BP);
-    const size_t fixed = 1024 /*align slack*/ + (4 * kMaxStages + 8) * 8 + sizeof(VecSmem) + 64;
+    const size_t sbytes = stage_bytes_for(BP);
+    P.nacc = std::min(kMaxAcc, kTmemCols / (4 * BP));
+    const size_t fixed = 1024 /*alignment slack*/ + (2 * kMaxStages + 2 * kMaxAcc + 2) * 8 + sizeof(VecSmem) +
+                         (size_t)fs.max_tiles_per_cta * sizeof(TileEntry);
     const size_t budget = 227 * 1024;
-    int stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / sb);
-    if (stages < 2) return cudaErrorNotSupported;
+    if (fixed + 2 * sbytes > budget) return cudaErrorNotSupported;
+    int stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / sbytes);
+    if (fs.stages_override > 0) stages = std::min(stages, std::max(2, fs.stages_override));
     P.stages = stages;
-    P.stage_bytes = (int)sb;
-    const size_t smem = (size_t)stages * sb + fixed;
+    P.stage_bytes = (int)sbytes;
+    const size_t smem = (size_t)stages * sbytes + fixed;
 
     static std::mutex mu;
     static std::map<void *, size_t> configured;
