@@ -181,6 +181,46 @@ KDA_API int kda_decode_debug_copy(kda_handle h, int which, void *dst, size_t byt
 /* KDA_DECODE_ABI_VERSION of the loaded library. */
 KDA_API int kda_decode_abi_version(void);
 
+/*
+ * kda_decode_step_noalloc -- the same decode step for callers that may not
+ * allocate device memory.  The pages describe no such entry point; it is a
+ * deployment convenience of this library.  It serves runtimes that own all
+ * device memory themselves (a pre-reserved pool that no library may grow) and
+ * serving loops that cannot afford the implicit device synchronisation of
+ * cudaMalloc / cudaFree.  It takes no handle and allocates no device memory
+ * (it calls no cudaMalloc, cudaFree or allocating library).
+ *
+ * It runs the five-kernel (KDA_ENGINE_SIMPLE) path, whatever cfg->engine says,
+ * with its fp32 activations in one file-scope device array of
+ * KDA_NOALLOC_MAX_SCRATCH_BYTES per device.  The activations of `batch`
+ * sequences take batch * (3 nh dk + 2 nh dv + nh + r) * 4 bytes, each of the
+ * seven arrays rounded up to 256 bytes; a step that needs more is rejected
+ * with KDA_ERR_UNSUPPORTED_SHAPE before anything is enqueued (for example
+ * batch 12 at hidden 4096, 32 heads of 128 x 128, r 64 fits; batch 64 at
+ * 48 heads of 128 x 128 does not).  Every stage writes its whole output
+ * before the next reads it, so nothing in the array needs to start at zero
+ * and nothing is cleared.
+ *
+ *   cfg          shape and out dtype as for kda_decode_init (validated the
+ *                same way; max_batch and engine are not used)
+ *   x, w, state_inout, out   as for kda_decode_step (device memory)
+ *   batch        1 .. any, within the scratch limit above
+ *   cuda_stream  cudaStream_t passed as void* (NULL = legacy default stream)
+ *
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's device address (cudaGetSymbolAddress, which may also load the
+ * library's device code on that device) and caches it; later calls only
+ * read the cache.  Make that first call before any stream capture begins.
+ *
+ * All calls on one device share the one array: two calls that can run at the
+ * same time (on different streams, or from host threads without ordering)
+ * race on it and corrupt each other's activations.  Order them (one stream,
+ * or events).  The set-up itself is thread-safe.
+ */
+#define KDA_NOALLOC_MAX_SCRATCH_BYTES (1u << 20)
+KDA_API int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weights *w, float *state_inout,
+                                    void *out, int batch, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,9 @@ EXPORTS = (
     "kda_decode_init", "kda_decode_set_stream", "kda_decode_step", "kda_decode_step_host", "kda_decode_sync",
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
+    "kda_decode_step_noalloc",
 )
+KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
 KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
 
 
@@ -88,6 +90,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_decode_last_error": (ctypes.c_char_p, [P]),
         "kda_decode_abi_version": (I, []),
         "kda_decode_debug_copy": (I, [P, I, P, ctypes.c_size_t]),
+        "kda_decode_step_noalloc": (I, [ctypes.POINTER(kda_config), P, ctypes.POINTER(kda_weights), P, P, I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -146,6 +149,12 @@ def kda_decode_scratch_bytes(cfg: kda_config) -> int:
 
 def kda_decode_debug_copy(h: int, which: int, dst: int, nbytes: int) -> None:
     _check(load().kda_decode_debug_copy(h, which, dst, nbytes), "kda_decode_debug_copy", h)
+
+
+def kda_decode_step_noalloc(cfg: kda_config, x: int, w: kda_weights, state: int, out: int, batch: int,
+                            stream: int) -> None:
+    _check(load().kda_decode_step_noalloc(ctypes.byref(cfg), x, ctypes.byref(w), state, out, batch, stream),
+           "kda_decode_step_noalloc")
 
 
 def kda_status_string(status: int) -> str:

@@ -2,6 +2,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 #include <string>
 
@@ -158,9 +159,87 @@ int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state
     return KDA_OK;
 }
 
+// ---------------------------------------------------------------- no-alloc entry point
+
+// The only device memory kda_decode_step_noalloc uses besides the caller's buffers: one
+// fixed array per device, for callers that may not allocate (see the header).
+__device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_MAX_SCRATCH_BYTES];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kNoAllocMaxDevices];  // device address of the array, per device (set-up cache)
+
+// Activations of `batch` sequences inside the array (same order as a handle's scratch);
+// returns false if they do not fit.
+bool noalloc_layout(const kda_config &c, int batch, char *base, kda::Scratch *s)
+{
+    const size_t B = (size_t)batch, Dk = (size_t)c.num_heads * c.head_dk, Dv = (size_t)c.num_heads * c.head_dv;
+    const size_t sizes[7] = {B * Dk * 4, B * Dk * 4, B * Dk * 4, B * Dv * 4, B * Dv * 4,
+                             B * (size_t)c.num_heads * 4, B * (size_t)c.alpha_rank * 4};
+    float **dst[7] = {&s->q, &s->k, &s->z, &s->v, &s->o, &s->bpre, &s->t};
+    size_t off = 0;
+    for (int i = 0; i < 7; ++i) {
+        if (off + sizes[i] > KDA_NOALLOC_MAX_SCRATCH_BYTES) return false;
+        *dst[i] = reinterpret_cast<float *>(base + off);
+        off += align_up(sizes[i], 256);
+    }
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
+
+int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weights *w, float *state_inout,
+                            void *out, int batch, void *cuda_stream)
+{
+    std::string why;
+    int rc = validate_config(cfg, &why);
+    if (rc) return rc;
+    if (batch < 1) return KDA_ERR_INVALID_ARG;
+    if (!x || !state_inout || !out) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(state_inout) || !aligned16(out)) return KDA_ERR_INVALID_ARG;
+    rc = check_weights(nullptr, w);
+    if (rc) return rc;
+    const size_t nx = (size_t)batch * cfg->hidden * 2;
+    const size_t ns = (size_t)batch * cfg->num_heads * cfg->head_dk * cfg->head_dv * 4;
+    const size_t no = (size_t)batch * cfg->hidden * (cfg->out_dtype == KDA_OUT_BF16 ? 2 : 4);
+    if (overlaps(state_inout, ns, x, nx) || overlaps(state_inout, ns, out, no)) return KDA_ERR_INVALID_ARG;
+    kda::Scratch s;
+    if (!noalloc_layout(*cfg, batch, nullptr, &s)) return KDA_ERR_UNSUPPORTED_SHAPE;  // over the fixed limit
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return KDA_ERR_NO_DEVICE; }
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return KDA_ERR_NO_DEVICE;
+    void *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {  // set-up, once per device, with that device current
+            int major = 0;
+            if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+                (void)cudaGetLastError();
+                return KDA_ERR_NO_DEVICE;
+            }
+            void *p = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess || !p) {
+                (void)cudaGetLastError();
+                return KDA_ERR_CUDA;
+            }
+            g_noalloc_ptr[dev] = p;
+        }
+        base = g_noalloc_ptr[dev];
+    }
+    noalloc_layout(*cfg, batch, static_cast<char *>(base), &s);
+    const kda::Dims d = dims_of(*cfg, batch);
+    const cudaError_t e = kda::simple_step(d, *w, x, state_inout, out, cfg->out_dtype, s,
+                                           static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
 
 int kda_decode_abi_version(void) { return KDA_DECODE_ABI_VERSION; }
 
