@@ -336,9 +336,8 @@ def kernel_rev() -> str:
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_attention_layer_kda_b200", "csrc")
-    for n in sorted(os.listdir(d)):
-        if n.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(d, n), "rb").read())
+    for n in ("common.cuh", "sm100.cuh", "fused.cuh", "fused.cu", "simple.cu"):  # the engines' kernels
+        h.update(open(os.path.join(d, n), "rb").read())
     return h.hexdigest()[:16]
 
 
