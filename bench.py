@@ -174,6 +174,35 @@ def run_reference(args, shape, rank):
     return 0
 
 
+def rank_inputs(shape: I.KdaShape, rank: int, world: int):
+    """Inputs of one rank: weights shared by all ranks; x and state are this rank's own
+    sequences, rows rank*B .. rank*B + B - 1 of the job's counter-based streams, so the N
+    ranks together hold exactly the sequences of one batch of N*B (data parallel, no
+    collective on the data path)."""
+    inp = I.generate(shape.replace(steps=1))
+    if world > 1:
+        B = shape.batch
+        inp.x[0] = I.gen_x(shape, 0, batch=B, row0=rank * B)
+        inp.state0 = I.gen_state(shape, batch=B, row0=rank * B)
+    return inp
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_steps_per_s(ms_per_step_slowest: float, world: int) -> float:
+    """Whole-job decode steps/s: every rank advances its own batch once per step."""
+    return world * 1000.0 / ms_per_step_slowest
+
+
 def workload_config(shape, n, l2_note):
     return {"workload": shape.name, "batch_per_gpu": shape.batch, "global_batch": shape.batch * n,
             "hidden": shape.hidden, "num_heads": shape.num_heads, "head_dk": shape.head_dk,
@@ -200,10 +229,7 @@ def run_ours(args, shape, rank, world, local_rank):
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
 
-    inp = I.generate(shape.replace(steps=1))
-    if world > 1:  # this rank's own sequences: the next rows of the same counter-based streams
-        inp.x[0] = I.gen_x(shape, 0, batch=B, row0=rank * B)
-        inp.state0 = I.gen_state(shape, batch=B, row0=rank * B)
+    inp = rank_inputs(shape, rank, world)
     set_bytes = ideal_bytes(shape, B)
     R = max(2, math.ceil(2 * l2 / set_bytes))
     wts = [tensors.to_device_weights(inp, dev) for _ in range(R)]
@@ -254,28 +280,25 @@ def run_ours(args, shape, rank, world, local_rank):
     ms_total = ev0.elapsed_time(ev1)
     clocks = clk.stop() if clk else None
 
-    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_per_step = ms_total / args.steps
-    steps_per_s_gpu = 1000.0 / ms_per_step
-    value = steps_per_s_gpu * world
+    value = job_steps_per_s(ms_per_step, world)
 
-    # end to end through the host-buffer entry point: H2D x, step, D2H out, sync, every step
-    e2e = None
-    if rank == 0:
-        xh = torch.from_numpy(inp.x[0].view(np.int16)).view(torch.bfloat16).pin_memory()
-        oh = torch.empty(B, shape.hidden, dtype=torch.float32).pin_memory()
-        n_e2e = args.e2e_steps if args.e2e_steps > 0 else max(10, min(args.steps, 2000))
-        for i in range(3):
-            dec.step_host(xh, ws[i % R], states[i % R], oh)
-        t0 = time.perf_counter()
-        for i in range(n_e2e):
-            dec.step_host(xh, ws[i % R], states[i % R], oh)
-        dt = time.perf_counter() - t0
-        e2e = {"value": world * n_e2e / dt, "unit": "steps/s", "h2d_bytes_per_step": int(xh.numel() * 2),
-               "d2h_bytes_per_step": int(oh.numel() * 4), "steps": n_e2e}
+    # end to end through the host-buffer entry point: H2D x, step, D2H out, sync, every step,
+    # on every rank; the slowest rank's wall time sets the job's rate
+    xh = torch.from_numpy(inp.x[0].view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty(B, shape.hidden, dtype=torch.float32).pin_memory()
+    n_e2e = args.e2e_steps if args.e2e_steps > 0 else max(10, min(args.steps, 2000))
+    for i in range(3):
+        dec.step_host(xh, ws[i % R], states[i % R], oh)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(n_e2e):
+        dec.step_host(xh, ws[i % R], states[i % R], oh)
+    dt = max_over_ranks(time.perf_counter() - t0, world, dev)
+    e2e = {"value": job_steps_per_s(1000.0 * dt / n_e2e, world), "unit": "steps/s",
+           "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 4), "steps": n_e2e}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
