@@ -143,6 +143,41 @@ KDA_API int kda_decode_step(kda_handle h, const void *x, const kda_weights *w, f
 KDA_API int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w, float *state_inout,
                          void *out_host, int batch);
 
+/*
+ * Several tokens per sequence in one call: `tokens` consecutive tokens of each of `batch`
+ * sequences, as in the verify step of multi-token (speculative) decoding that the Kiln post
+ * ("What did we measure that did not pay?") and the TileRT README (MTP) describe.
+ *   x            bf16 [batch * tokens, H]; row b * tokens + t is token t of sequence b
+ *   state_inout  fp32 [batch, nh, dk, dv]; advanced by `tokens` steps, token by token
+ *   out          [batch * tokens, H] (cfg.out_dtype); row b * tokens + t is the output of
+ *                token t, read out after token t's update
+ * The projections read the weights once for all batch * tokens rows.  Requires
+ * tokens >= 1 and batch * tokens <= max_batch.  tokens == 1 is kda_decode_step; more
+ * tokens run the five-kernel engine (KDA_ENGINE_SIMPLE kernels, one state kernel that
+ * applies the tokens in order).  The result equals `tokens` successive kda_decode_step
+ * calls on that engine bit for bit.  Same errors and ordering as kda_decode_step.
+ */
+KDA_API int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out,
+                                   int batch, int tokens);
+
+/*
+ * Recurrent-state checkpoint and restore (the Kiln post's prefix cache keeps checkpoints of
+ * linear-attention state in a host tier: "What is Kiln?"; its "What could only a device
+ * show?" is the lesson that such a copy must be ordered behind the queued work).  Both are
+ * enqueued on the handle's stream, after every step enqueued before them and before every
+ * step enqueued after them, so a checkpoint holds exactly the state those steps produced
+ * and a restore is what the next step reads.
+ *   state     device fp32 [*, nh, dk, dv] (the state_inout of the steps)
+ *   seq0, nseq  sequences [seq0, seq0 + nseq): seq0 >= 0, nseq >= 1, seq0 + nseq <=
+ *               max_batch, and inside the caller's state buffer
+ *   host      host memory of nseq * nh * dk * dv * 4 bytes, sequence-major (page-locked
+ *             memory makes the copy asynchronous; pageable memory makes the call wait)
+ * The host buffer must not be read (checkpoint) or reused (restore) before the stream has
+ * passed the copy: kda_decode_sync(h) or any later wait on the stream.
+ */
+KDA_API int kda_state_checkpoint(kda_handle h, const float *state, int seq0, int nseq, void *host_dst);
+KDA_API int kda_state_restore(kda_handle h, const void *host_src, float *state, int seq0, int nseq);
+
 /* Waits for the handle's stream; returns the device status of the steps since
  * the last check (KDA_OK or KDA_ERR_DEVICE_TIMEOUT) and clears it. */
 KDA_API int kda_decode_sync(kda_handle h);

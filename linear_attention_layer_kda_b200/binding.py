@@ -33,7 +33,7 @@ EXPORTS = (
     "kda_decode_init", "kda_decode_set_stream", "kda_decode_step", "kda_decode_step_host", "kda_decode_sync",
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
-    "kda_decode_step_noalloc",
+    "kda_decode_step_noalloc", "kda_decode_step_tokens", "kda_state_checkpoint", "kda_state_restore",
 )
 KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
 KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
@@ -91,6 +91,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_decode_abi_version": (I, []),
         "kda_decode_debug_copy": (I, [P, I, P, ctypes.c_size_t]),
         "kda_decode_step_noalloc": (I, [ctypes.POINTER(kda_config), P, ctypes.POINTER(kda_weights), P, P, I, P]),
+        "kda_decode_step_tokens": (I, [P, P, ctypes.POINTER(kda_weights), P, P, I, I]),
+        "kda_state_checkpoint": (I, [P, P, I, I, P]),
+        "kda_state_restore": (I, [P, P, P, I, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -119,6 +122,18 @@ def kda_decode_set_stream(h: int, stream: int) -> None:
 
 def kda_decode_step(h: int, x: int, w: kda_weights, state: int, out: int, batch: int) -> None:
     _check(load().kda_decode_step(h, x, ctypes.byref(w), state, out, batch), "kda_decode_step", h)
+
+
+def kda_decode_step_tokens(h: int, x: int, w: kda_weights, state: int, out: int, batch: int, tokens: int) -> None:
+    _check(load().kda_decode_step_tokens(h, x, ctypes.byref(w), state, out, batch, tokens), "kda_decode_step_tokens", h)
+
+
+def kda_state_checkpoint(h: int, state: int, seq0: int, nseq: int, host_dst: int) -> None:
+    _check(load().kda_state_checkpoint(h, state, seq0, nseq, host_dst), "kda_state_checkpoint", h)
+
+
+def kda_state_restore(h: int, host_src: int, state: int, seq0: int, nseq: int) -> None:
+    _check(load().kda_state_restore(h, host_src, state, seq0, nseq), "kda_state_restore", h)
 
 
 def kda_decode_step_host(h: int, x_host: int, w: kda_weights, state: int, out_host: int, batch: int) -> None:
@@ -221,6 +236,26 @@ class KdaDecoder:
         b = x_host.shape[0] if batch is None else batch
         self._bind_stream()
         kda_decode_step_host(self.h, x_host.data_ptr(), weights, state.data_ptr(), out_host.data_ptr(), b)
+
+    def step_tokens(self, x, weights: kda_weights, state, out, batch: int, tokens: int) -> None:
+        """`tokens` tokens of each of `batch` sequences; x and out are [batch * tokens, H]."""
+        for n, a in (("x", x), ("state", state), ("out", out)):
+            if not a.is_cuda or not a.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous CUDA tensor")
+        self._bind_stream()
+        kda_decode_step_tokens(self.h, x.data_ptr(), weights, state.data_ptr(), out.data_ptr(), batch, tokens)
+
+    def checkpoint(self, state, host, seq0: int = 0, nseq: Optional[int] = None) -> None:
+        """Enqueues a copy of sequences [seq0, seq0 + nseq) of `state` into the host tensor `host`."""
+        n = state.shape[0] - seq0 if nseq is None else nseq
+        self._bind_stream()
+        kda_state_checkpoint(self.h, state.data_ptr(), seq0, n, host.data_ptr())
+
+    def restore(self, host, state, seq0: int = 0, nseq: Optional[int] = None) -> None:
+        """Enqueues a copy of the host tensor `host` into sequences [seq0, seq0 + nseq) of `state`."""
+        n = state.shape[0] - seq0 if nseq is None else nseq
+        self._bind_stream()
+        kda_state_restore(self.h, host.data_ptr(), state.data_ptr(), seq0, n)
 
     def sync(self) -> None:
         kda_decode_sync(self.h)

@@ -394,6 +394,59 @@ int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w,
     return take_device_status(h);
 }
 
+int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out,
+                           int batch, int tokens)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    if (tokens < 1) return fail(h, KDA_ERR_INVALID_ARG, "tokens must be >= 1");
+    if (tokens == 1) return kda_decode_step(h, x, w, state_inout, out, batch);
+    if (batch < 1 || (long long)batch * tokens > h->cfg.max_batch)
+        return fail(h, KDA_ERR_INVALID_ARG, "batch * tokens must be in [1, max_batch]");
+    if (!x || !state_inout || !out) return fail(h, KDA_ERR_INVALID_ARG, "null x, state or out");
+    if (!aligned16(x) || !aligned16(state_inout) || !aligned16(out))
+        return fail(h, KDA_ERR_INVALID_ARG, "x, state and out must be 16-byte aligned");
+    int rc = check_weights(h, w);
+    if (rc) return rc;
+    const kda_config &c = h->cfg;
+    const size_t rows = (size_t)batch * tokens;
+    const size_t nx = rows * c.hidden * 2, no = rows * c.hidden * (c.out_dtype == KDA_OUT_BF16 ? 2 : 4);
+    const size_t ns = (size_t)batch * c.num_heads * c.head_dk * c.head_dv * 4;
+    if (overlaps(state_inout, ns, x, nx) || overlaps(state_inout, ns, out, no))
+        return fail(h, KDA_ERR_INVALID_ARG, "state_inout overlaps x or out");
+    rc = take_device_status(h);
+    if (rc) return rc;
+    const cudaError_t e = kda::simple_step_tokens(dims_of(c, batch), tokens, *w, x, state_inout, out, c.out_dtype,
+                                                  h->s, h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
+    return KDA_OK;
+}
+
+static int state_copy(kda_handle h, void *dst, const void *src, int seq0, int nseq, bool to_host)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    if (!dst || !src) return fail(h, KDA_ERR_INVALID_ARG, "null state or host buffer");
+    if (seq0 < 0 || nseq < 1 || (long long)seq0 + nseq > h->cfg.max_batch)
+        return fail(h, KDA_ERR_INVALID_ARG, "need seq0 >= 0, nseq >= 1 and seq0 + nseq <= max_batch");
+    const kda_config &c = h->cfg;
+    const size_t per_seq = (size_t)c.num_heads * c.head_dk * c.head_dv * 4;
+    const size_t off = (size_t)seq0 * per_seq, n = (size_t)nseq * per_seq;
+    const cudaError_t e =
+        to_host ? cudaMemcpyAsync(dst, static_cast<const char *>(src) + off, n, cudaMemcpyDeviceToHost, h->stream)
+                : cudaMemcpyAsync(static_cast<char *>(dst) + off, src, n, cudaMemcpyHostToDevice, h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, to_host ? "state checkpoint copy" : "state restore copy");
+    return KDA_OK;
+}
+
+int kda_state_checkpoint(kda_handle h, const float *state, int seq0, int nseq, void *host_dst)
+{
+    return state_copy(h, host_dst, state, seq0, nseq, true);
+}
+
+int kda_state_restore(kda_handle h, const void *host_src, float *state, int seq0, int nseq)
+{
+    return state_copy(h, state, host_src, seq0, nseq, false);
+}
+
 int kda_decode_sync(kda_handle h)
 {
     if (!h) return KDA_ERR_INVALID_ARG;

@@ -36,6 +36,10 @@ struct Dims {
 cudaError_t simple_step(const Dims &d, const kda_weights &w, const void *x, float *state, void *out,
                         int out_dtype, const Scratch &s, cudaStream_t stream);
 int simple_launches();
+// `tokens` consecutive tokens of each of d.B sequences (x, out: [d.B * tokens, H], row
+// b*tokens + t); the state advances token by token.
+cudaError_t simple_step_tokens(const Dims &d, int tokens, const kda_weights &w, const void *x, float *state,
+                               void *out, int out_dtype, const Scratch &s, cudaStream_t stream);
 
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__

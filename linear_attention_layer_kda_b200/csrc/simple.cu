@@ -197,18 +197,71 @@ __global__ void __launch_bounds__(DV)
     o[(size_t)b * nh * DV + (size_t)h * DV + j] = fmaf(u, kq, p);
 }
 
+// Several consecutive tokens of one sequence: one block per (head, sequence) runs the
+// single-token update above once per token, in token order, on the same state column.
+// Row b*T + t of the activations is token t of sequence b; o row b*T + t is the readout
+// after token t.  Thread j only ever touches column j of S, so the in-place updates of
+// consecutive tokens need no synchronisation beyond the shared vectors' reloads.
+template <int DK, int DV>
+__global__ void __launch_bounds__(DV)
+    k_state_tokens(const float *__restrict__ q, const float *__restrict__ k, const float *__restrict__ v,
+                   const float *__restrict__ bpre, const float *__restrict__ z, float *__restrict__ state,
+                   float *__restrict__ o, int nh, int T)
+{
+    __shared__ float s_q[DK], s_k[DK], s_a[DK];
+    const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
+    float *S = state + ((size_t)b * nh + h) * DK * DV;
+    for (int t = 0; t < T; ++t) {
+        const size_t row = (size_t)b * T + t;
+        const size_t hk = row * nh * DK + (size_t)h * DK;
+        __syncthreads();  // the previous token's readers of s_q, s_k, s_a are done
+        for (int i = j; i < DK; i += DV) {
+            s_q[i] = q[hk + i];
+            s_k[i] = k[hk + i];
+            s_a[i] = 1.f / (1.f + expf(z[hk + i]));  // exp(-softplus(z)) = sigmoid(-z)
+        }
+        __syncthreads();
+        float ss = 0.f;
+        for (int i = 0; i < DK; ++i) ss = fmaf(s_k[i], s_k[i], ss);
+        const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+        __syncthreads();
+        for (int i = j; i < DK; i += DV) s_k[i] *= inv;
+        __syncthreads();
+        const float beta = 1.f / (1.f + expf(-bpre[row * nh + h]));
+        float w = 0.f, p = 0.f, kq = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < DK; ++i) {
+            const float st = s_a[i] * S[(size_t)i * DV + j];
+            w = fmaf(s_k[i], st, w);
+            p = fmaf(s_q[i], st, p);
+            kq = fmaf(s_k[i], s_q[i], kq);
+        }
+        const float u = beta * (v[row * nh * DV + (size_t)h * DV + j] - w);
+#pragma unroll 8
+        for (int i = 0; i < DK; ++i) {
+            float *e = S + (size_t)i * DV + j;
+            *e = fmaf(s_k[i], u, s_a[i] * *e);
+        }
+        o[row * nh * DV + (size_t)h * DV + j] = fmaf(u, kq, p);
+    }
+}
+
 template <int DK, int DV>
 void launch_state(const Dims &d, const Scratch &s, float *state, cudaStream_t st)
 {
     k_state<DK, DV><<<dim3(d.nh, d.B), DV, 0, st>>>(s.q, s.k, s.v, s.bpre, s.z, state, s.o, d.nh);
 }
 
-}  // namespace
+template <int DK, int DV>
+void launch_state_tokens(const Dims &d, int nseq, int T, const Scratch &s, float *state, cudaStream_t st)
+{
+    k_state_tokens<DK, DV><<<dim3(d.nh, nseq), DV, 0, st>>>(s.q, s.k, s.v, s.bpre, s.z, state, s.o, d.nh, T);
+}
 
-int simple_launches() { return 5; }
-
-cudaError_t simple_step(const Dims &d, const kda_weights &w, const void *x, float *state, void *out,
-                        int out_dtype, const Scratch &s, cudaStream_t st)
+// The five stages for d.B activation rows; the state stage covers nseq sequences of T
+// tokens each (d.B = nseq * T; T == 1 is the single-token step).
+cudaError_t simple_run(const Dims &d, int nseq, int T, const kda_weights &w, const void *x, float *state,
+                       void *out, int out_dtype, const Scratch &s, cudaStream_t st)
 {
     const int H = d.H, Dk = d.Dk(), Dv = d.Dv();
     const int by = (d.B + kBatchChunk - 1) / kBatchChunk;
@@ -238,10 +291,17 @@ cudaError_t simple_step(const Dims &d, const kda_weights &w, const void *x, floa
         k_gemv_bf16<float><<<dim3((Dk + 7) / 8, by, 1), 256, 0, st>>>(jz, jz, d.r, s.t, d.B);
     }
     // 4. state update and readout
-    if (d.dk == 128 && d.dv == 128) launch_state<128, 128>(d, s, state, st);
-    else if (d.dk == 64 && d.dv == 64) launch_state<64, 64>(d, s, state, st);
-    else if (d.dk == 128 && d.dv == 64) launch_state<128, 64>(d, s, state, st);
-    else launch_state<64, 128>(d, s, state, st);
+    if (T == 1) {
+        if (d.dk == 128 && d.dv == 128) launch_state<128, 128>(d, s, state, st);
+        else if (d.dk == 64 && d.dv == 64) launch_state<64, 64>(d, s, state, st);
+        else if (d.dk == 128 && d.dv == 64) launch_state<128, 64>(d, s, state, st);
+        else launch_state<64, 128>(d, s, state, st);
+    } else {
+        if (d.dk == 128 && d.dv == 128) launch_state_tokens<128, 128>(d, nseq, T, s, state, st);
+        else if (d.dk == 64 && d.dv == 64) launch_state_tokens<64, 64>(d, nseq, T, s, state, st);
+        else if (d.dk == 128 && d.dv == 64) launch_state_tokens<128, 64>(d, nseq, T, s, state, st);
+        else launch_state_tokens<64, 128>(d, nseq, T, s, state, st);
+    }
     // 5. out = W_o o
     {
         ProjJob jo{w.wo, w.so, nullptr};
@@ -253,6 +313,24 @@ cudaError_t simple_step(const Dims &d, const kda_weights &w, const void *x, floa
                                                                               static_cast<float *>(out));
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+int simple_launches() { return 5; }
+
+cudaError_t simple_step(const Dims &d, const kda_weights &w, const void *x, float *state, void *out,
+                        int out_dtype, const Scratch &s, cudaStream_t st)
+{
+    return simple_run(d, d.B, 1, w, x, state, out, out_dtype, s, st);
+}
+
+cudaError_t simple_step_tokens(const Dims &d, int tokens, const kda_weights &w, const void *x, float *state,
+                               void *out, int out_dtype, const Scratch &s, cudaStream_t st)
+{
+    Dims rows = d;
+    rows.B = d.B * tokens;
+    return simple_run(rows, d.B, tokens, w, x, state, out, out_dtype, s, st);
 }
 
 }  // namespace kda
