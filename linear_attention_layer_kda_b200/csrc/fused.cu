@@ -49,10 +49,16 @@ constexpr int kThreads = 512;
 constexpr int kMaxBP = 64;
 constexpr int kTileBytes = 128 * 128;
 constexpr int kHeadsPerGroup = 8;
+// Head groups of q/k/v tiles between a group's q/k/v tiles and its W_o tiles (-1: all W_o
+// tiles after all q/k/v tiles).  Measured at batch 8: interleaving (1, 2, 3) stalls the MMA on
+// o blocks whose state units are still running, so the default keeps W_o last.
+constexpr int kWoLag = -1;
 constexpr int kMaxStages = 12;   // ring stages (weight tile + activation planes)
 constexpr int kMaxAcc = 8;       // TMEM accumulator buffers
 constexpr int kMaxTilesPerCta = 512;
 constexpr int kTmemCols = 512;
+constexpr int kEarlyTiles = 2;                 // weight copies issued before x is known final
+constexpr uint64_t kEarlyHoldNs = 6000;        // longest hold of the rest of the stream
 
 // Optional timeline (compile with -DKDA_TRACE): per CTA, kTraceSlots global-timer stamps.
 #ifdef KDA_TRACE
@@ -75,19 +81,19 @@ enum TraceSlot {
 // counters (uint32, monotonic across steps; targets are multiples of the step count)
 //   C_XQ          x K-blocks split into planes (B per K block per step)
 //   C_GATE        gate rows finished
-//   C_CLAIM0/1    state-unit claim counter of even / odd steps
+//   C_CLAIM0/1    (unused: state units are assigned statically)
 //   C_ABORT       set by any wait that gives up
 //   off_oready+kb state units done for o K-block kb (B per step)
 //   off_rb+key    segments published for row block key (q, k, v, o row blocks)
 constexpr int C_XQ = 0, C_GATE = 1, C_CLAIM0 = 2, C_ABORT = 4, C_FIXED = 16;
 
 struct __align__(16) VecSmem {
-    float q[256], k[256], a[256];  // per head of the unit: q, k^, alpha  (heads_per_unit * dk)
+    float q[256], k[256];          // per head of the unit: q, k^  (heads_per_unit * dk)
+    float a[2][256];               // alpha of the current and the next unit (by unit parity)
     float v[128], u[128], o[128];  // per virtual column of the unit
-    float t[256];                  // W_a_down x of the unit's sequence
     float red_w[8][128], red_p[8][128];
-    float beta[2], kq[2], inv[2];
-    int unit, ok;
+    float beta[2][2], kq[2], inv[2];  // beta: [unit parity][head of the unit]
+    int unit, ok, fail;
 };
 
 struct FusedParams {
@@ -210,6 +216,35 @@ __device__ __forceinline__ float sum_partials(const FusedParams &P, int key, int
         for (int g = 0; g < 8; ++g) s += v[g];
     }
     return s;
+}
+
+// Two sums of the kind above with all their loads issued together (8 slots per item at a
+// time); items with has[j] false are skipped.  Same slot order, so the same bits.
+template <int BP>
+__device__ __forceinline__ void sum_partials2(const FusedParams &P, const int (&key)[2], const int (&r)[2],
+                                              const bool (&has)[2], int b, float (&out)[2])
+{
+    uint2 info[2];
+    const float *base[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        info[j] = has[j] ? __ldg(P.rbinfo + key[j]) : make_uint2(0u, 0u);
+        base[j] = P.part + ((size_t)info[j].x * BP + b) * 128 + r[j];
+        out[j] = 0.f;
+    }
+    const uint32_t nmax = info[0].y > info[1].y ? info[0].y : info[1].y;
+    for (uint32_t g0 = 0; g0 < nmax; g0 += 8) {
+        float v[2][8];
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                v[j][g] = g0 + g < info[j].y ? __ldcg(base[j] + (size_t)(g0 + g) * BP * 128) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int g = 0; g < 8; ++g) out[j] += v[j][g];
+    }
 }
 
 __device__ __forceinline__ bool wait_rb(const FusedParams &P, int key, const Ctl &c, int where)
@@ -372,10 +407,52 @@ __device__ void gate_rows(const FusedParams &P, VecSmem *vs, int vt)
     }
 }
 
-// One state unit: sequence b, o K-block kb (heads kb*128/dv ..), all dk rows.
-template <int BP, int DK>
-__device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int b, int kb, int vt, int nu)
+// Gates of state unit u (sequence u % B, o K-block u / B) into slot `slot`: beta of its
+// heads and alpha = exp(-softplus(z)) = 1 / (1 + e^z), z = W_a_up[row] . t, of its rows,
+// computed by vector threads [t0, t0 + nt).  t and W_b x must be final (C_GATE acquired).
+template <int DK>
+__device__ void unit_gates(const FusedParams &P, VecSmem *vs, int u, int slot, int vt, int t0, int nt)
 {
+    const int b = u % P.B, kb = u / P.B, hpu = 128 / P.dv, h0 = kb * hpu;
+    const int me = vt - t0;
+    if (me < 0 || me >= nt) return;
+    if (me < hpu) vs->beta[slot][me] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + me)));
+    const float *t = P.t + (size_t)b * P.r;
+    for (int i = me; i < hpu * DK; i += nt) {
+        const uint16_t *wr = P.wa_up + ((size_t)h0 * DK + i) * P.r;
+        float z = 0.f;
+        for (int j0 = 0; j0 < P.r; j0 += 32) {
+            uint4 w4[4];
+            float4 t4[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                w4[q] = j0 + q * 8 < P.r ? __ldg(reinterpret_cast<const uint4 *>(wr + j0 + q * 8)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                t4[q] = j0 + q * 4 < P.r ? __ldcg(reinterpret_cast<const float4 *>(t + j0 + q * 4)) : make_float4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t wv[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
+                const float tv[8] = {t4[2 * q].x, t4[2 * q].y, t4[2 * q].z, t4[2 * q].w,
+                                     t4[2 * q + 1].x, t4[2 * q + 1].y, t4[2 * q + 1].z, t4[2 * q + 1].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    z = fmaf(bf16_bits_to_float(wv[e] & 0xFFFFu), tv[2 * e], z);
+                    z = fmaf(bf16_bits_to_float(wv[e] >> 16), tv[2 * e + 1], z);
+                }
+            }
+        }
+        vs->a[slot][i] = 1.f / (1.f + expf(z));
+    }
+}
+
+// One state unit: sequence b, o K-block kb (heads kb*128/dv ..), all dk rows.  Its gates are
+// in slot nu & 1; while warp 0 waits for the unit's q/k/v, warps 1-7 compute the gates of
+// this CTA's next unit (next_u >= 0) into the other slot.
+template <int BP, int DK>
+__device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int u, int next_u, int vt, int nu)
+{
+    const int b = u % P.B, kb = u / P.B, slot = nu & 1;
     constexpr int RPW = DK / 8;  // rows per warp
     const int vw = vt >> 5, lane = vt & 31;
     const int dv = P.dv, hpu = 128 / dv, h0 = kb * hpu;
@@ -387,62 +464,56 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 #pragma unroll
     for (int r = 0; r < RPW; ++r) s[r] = ld_stream_f4(S + (size_t)(vw * RPW + r) * dv);
 
-    // gates first: t and W_b x are final long before the unit's heads
-    if (vt == 0) vs->ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);
+    if (vt == 0) vs->fail = 0;
     named_bar(2, 256);
-    if (!vs->ok) return false;
-    for (int j = vt; j < P.r; j += 256) vs->t[j] = __ldcg(P.t + (size_t)b * P.r + j);
-    if (vt < hpu) vs->beta[vt] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + vt)));
+    // then the heads' q, k, v: wait for every segment of their row blocks (one thread per
+    // counter, so the round trips overlap), add the partials
+    {
+        const int rlo = h0 * DK / 128, nq = ((h0 + hpu) * DK - 1) / 128 - rlo + 1;
+        if (vt < 2 * nq + 1) {
+            const int key = vt < nq ? rlo + vt : (vt < 2 * nq ? P.nRBq + rlo + (vt - nq) : 2 * P.nRBq + kb);
+            if (!wait_rb(P, key, c, 11)) vs->fail = 1;
+        }
+        if (next_u >= 0) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
+    }
     named_bar(2, 256);
-    // alpha = exp(-softplus(z)) = 1 / (1 + e^z),  z = W_a_up[row] . t
-    for (int i = vt; i < hpu * DK; i += 256) {
-        const uint16_t *wr = P.wa_up + ((size_t)h0 * DK + i) * P.r;
-        float z = 0.f;
-        for (int j0 = 0; j0 < P.r; j0 += 64) {
-            uint4 w8[8];
-#pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8)
-                w8[q8] = j0 + q8 * 8 < P.r ? __ldg(reinterpret_cast<const uint4 *>(wr + j0 + q8 * 8)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8) {
-                const uint32_t wv[4] = {w8[q8].x, w8[q8].y, w8[q8].z, w8[q8].w};
-                const int j = j0 + q8 * 8;
-                if (j < P.r) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        z = fmaf(bf16_bits_to_float(wv[e] & 0xFFFFu), vs->t[j + 2 * e], z);
-                        z = fmaf(bf16_bits_to_float(wv[e] >> 16), vs->t[j + 2 * e + 1], z);
-                    }
+    if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
+    if (vs->fail) return false;
+    {
+        // items: q and k rows of the unit's heads, then its 128 v columns; a thread's items
+        // are loaded together (one memory round trip), then summed in slot order
+        const int nqk = hpu * DK, nitems = 2 * nqk + 128;
+        for (int it0 = 0; it0 < nitems; it0 += 512) {  // 384 items (dk = 128) or 640 (dk = 128, dv = 64)
+            int key[2], r[2];
+            bool has[2];
+    #pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int it = it0 + vt + 256 * j;
+                has[j] = it < nitems;
+                if (it < 2 * nqk) {
+                    const int row = h0 * DK + it % nqk;
+                    key[j] = (it / nqk) * P.nRBq + row / 128;
+                    r[j] = row % 128;
+                } else {
+                    key[j] = 2 * P.nRBq + kb;
+                    r[j] = it - 2 * nqk;
                 }
             }
-        }
-        vs->a[i] = 1.f / (1.f + expf(z));
-    }
-    // then the heads' q, k, v: wait for every segment of their row blocks, add the partials
-    if (vt == 0) {
-        bool ok = true;
-        const int rlo = h0 * DK / 128, rhi = ((h0 + hpu) * DK - 1) / 128;
-        for (int rb = rlo; ok && rb <= rhi; ++rb) ok = wait_rb(P, rb, c, 11) && wait_rb(P, P.nRBq + rb, c, 11);
-        if (ok) ok = wait_rb(P, 2 * P.nRBq + kb, c, 11);
-        vs->ok = ok;
-        if (nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
-    }
-    named_bar(2, 256);
-    if (!vs->ok) return false;
-    {
-        const int nqk = hpu * DK;
-        for (int it = vt; it < 2 * nqk + 128; it += 256) {
-            if (it < 2 * nqk) {
-                const int i = it % nqk, isk = it / nqk;
-                const int row = h0 * DK + i;
-                const float val = sum_partials<BP>(P, isk * P.nRBq + row / 128, b, row % 128);
-                (isk ? vs->k : vs->q)[i] = val;
-                (isk ? P.k : P.q)[(size_t)b * Dk + row] = val;  // kept for kda_decode_debug_copy
-            } else {
-                const int i = it - 2 * nqk;
-                const float val = sum_partials<BP>(P, 2 * P.nRBq + kb, b, i);
-                vs->v[i] = val;
-                P.v[(size_t)b * Dv + (size_t)kb * 128 + i] = val;
+            float val[2];
+            sum_partials2<BP>(P, key, r, has, b, val);
+    #pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int it = it0 + vt + 256 * j;
+                if (!has[j]) continue;
+                if (it < 2 * nqk) {
+                    const int i = it % nqk, isk = it / nqk, row = h0 * DK + i;
+                    (isk ? vs->k : vs->q)[i] = val[j];
+                    (isk ? P.k : P.q)[(size_t)b * Dk + row] = val[j];  // kept for kda_decode_debug_copy
+                } else {
+                    const int i = it - 2 * nqk;
+                    vs->v[i] = val[j];
+                    P.v[(size_t)b * Dv + (size_t)kb * 128 + i] = val[j];
+                }
             }
         }
     }
@@ -472,7 +543,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 #pragma unroll
     for (int r = 0; r < RPW; ++r) {
         const int i = hh * DK + vw * RPW + r;
-        const float a = vs->a[i], kk = vs->k[i], qq = vs->q[i];
+        const float a = vs->a[slot][i], kk = vs->k[i], qq = vs->q[i];
         s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
         pw.x = fmaf(kk, s[r].x, pw.x); pw.y = fmaf(kk, s[r].y, pw.y);
         pw.z = fmaf(kk, s[r].z, pw.z); pw.w = fmaf(kk, s[r].w, pw.w);
@@ -490,9 +561,9 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
             p += vs->red_p[j][vt];
         }
         const int hx = vt / dv;
-        const float u = vs->beta[hx] * (vs->v[vt] - w);
-        vs->u[vt] = u;
-        vs->o[vt] = fmaf(u, vs->kq[hx], p);
+        const float uu = vs->beta[slot][hx] * (vs->v[vt] - w);
+        vs->u[vt] = uu;
+        vs->o[vt] = fmaf(uu, vs->kq[hx], p);
     }
     named_bar(2, 256);
     // o -> four E4M3 planes with one power-of-two scale for the K-block; release it
@@ -546,16 +617,24 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
                                       (uint32_t)(nb - o < 32768 ? nb - o : 32768), pol);
         }
     }
+    // State units (sequence u % B, o K-block u / B) in head order, CTA c taking c, c + grid,
+    // ...: the same units every step, so the next unit's gates are computed while the
+    // current one waits for its q/k/v.
     const int units = P.B * P.nKBo;
-    uint32_t *claim = P.ctr + C_CLAIM0 + (P.epoch & 1u);
-    for (int nu = 0;; ++nu) {
-        if (vt == 0) vs->unit = should_stop(c) ? units : (int)atomicAdd(claim, 1u);
+    if ((int)blockIdx.x < units) {
+        if (vt == 0) vs->ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);  // t and W_b x final
         named_bar(2, 256);
-        const int u = vs->unit;
+        if (!vs->ok) return;
+        unit_gates<DK>(P, vs, blockIdx.x, 0, vt, 0, 256);
         named_bar(2, 256);
-        if (u >= units) break;
+    }
+    for (int nu = 0, u = blockIdx.x; u < units; ++nu, u += gridDim.x) {
+        if (vt == 0) vs->unit = should_stop(c) ? 1 : 0;
+        named_bar(2, 256);
+        if (vs->unit) return;
         if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu);
-        if (!state_unit<BP, DK>(P, vs, c, u % P.B, u / P.B, vt, nu)) return;
+        const int next = u + (int)gridDim.x < units ? u + (int)gridDim.x : -1;
+        if (!state_unit<BP, DK>(P, vs, c, u, next, vt, nu)) return;
         if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
     }
     // out = sum of the W_o partials: items of (row block, 32-row quarter)
@@ -622,8 +701,18 @@ __device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *m
         fence_proxy_async_global();  // planes written by other SMs, read by the async proxy
         return true;
     };
+    // Hold the weight stream back after the first kEarlyTiles copies until x is split into
+    // planes (or kEarlyHoldNs passed): the x loads of the splitting CTAs then do not queue
+    // behind a full ring of weight copies from every SM, and the MMA starts sooner.
+    const uint64_t hold_until = globaltimer_ns() + kEarlyHoldNs;
     while (na < n) {
         bool progress = false;
+        if (!x_ok && nw >= kEarlyTiles && nw < n && my[nw].mat < 3 && globaltimer_ns() < hold_until) {
+            if (!poll_ready(my[nw])) {
+                __nanosleep(128);
+                continue;
+            }
+        }
         while (na < nw && known_ready(my[na])) {
             const TileEntry e = my[na];
             const int s = na % R.S;
@@ -825,7 +914,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
         }
         *sh_abort = 0;
         mbar_fence_init();
-        if (blockIdx.x == 0) P.ctr[C_CLAIM0 + ((P.epoch + 1u) & 1u)] = 0u;  // next step's unit counter
     }
     if (warp == 3 && lane == 0) {
         // small inputs every CTA reads soon: pull them into L2 before the weight stream queues up
@@ -955,7 +1043,10 @@ void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, s
 {
     const int nKBx = d.H / 128, nKBo = d.Dv() / 128, nRBq = d.Dk() / 128, nRBv = d.Dv() / 128, nRBo = d.H / 128;
     const int hpu = std::max(128 / d.dk, 128 / d.dv);
-    const int hpg = std::max(hpu, kHeadsPerGroup / hpu * hpu);
+    int heads_per_group = kHeadsPerGroup, wo_lag = kWoLag;
+    if (const char *e = getenv("KDA_HEADS_PER_GROUP")) heads_per_group = std::max(1, atoi(e));
+    if (const char *e = getenv("KDA_WO_LAG")) wo_lag = atoi(e);
+    const int hpg = std::max(hpu, heads_per_group / hpu * hpu);
     const int G = (d.nh + hpg - 1) / hpg;
     struct T { uint8_t mat; uint16_t rb, kb; };
     std::vector<std::vector<T>> per_cta(P);
@@ -973,7 +1064,7 @@ void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, s
         for (int c = 0; c < P; ++c)
             for (size_t i = 0; i < len[c]; ++i) per_cta[c].push_back(list[pos++]);
     };
-    for (int g = 0; g < G; ++g) {
+    auto qkv_group = [&](int g) {
         const int h0 = g * hpg, h1 = std::min(d.nh, h0 + hpg);
         std::vector<T> list;
         for (int m = 0; m < 3; ++m) {
@@ -982,14 +1073,22 @@ void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, s
                 for (int kb = 0; kb < nKBx; ++kb) list.push_back(T{(uint8_t)m, (uint16_t)rb, (uint16_t)kb});
         }
         split(list);
-    }
-    for (int g = 0; g < G; ++g) {
+    };
+    auto wo_group = [&](int g) {
         const int h0 = g * hpg, h1 = std::min(d.nh, h0 + hpg);
         std::vector<T> list;
         for (int rb = 0; rb < nRBo; ++rb)
             for (int kb = h0 * d.dv / 128; kb < h1 * d.dv / 128; ++kb) list.push_back(T{3, (uint16_t)rb, (uint16_t)kb});
         split(list);
+    };
+    // The W_o tiles of group g follow the q/k/v tiles of group g + lag, so the state units of
+    // group g run while the weight stream carries later groups' q/k/v.
+    const int lag = wo_lag < 0 ? G : wo_lag;
+    for (int g = 0; g < G; ++g) {
+        qkv_group(g);
+        if (g - lag >= 0) wo_group(g - lag);
     }
+    for (int g = std::max(0, G - lag); g < G; ++g) wo_group(g);
     // row-block keys: q 0.., k nRBq.., v 2nRBq.., o 2nRBq+nRBv..
     auto key = [&](const T &t) {
         return t.mat == 3 ? 2 * nRBq + nRBv + t.rb : (t.mat == 2 ? 2 * nRBq + t.rb : t.mat * nRBq + t.rb);
