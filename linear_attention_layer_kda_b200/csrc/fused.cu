@@ -736,9 +736,9 @@ __device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *m
             continue;
         }
         const uint64_t now = globaltimer_ns();
-        if (na < nw && now >= t_poll) {  // a poll is a global round trip: at most one per 0.5 us
+        if (na < nw && now >= t_poll) {  // a poll is a global round trip: at most one per 0.2 us
             if (poll_ready(my[na])) progress = true;
-            else t_poll = globaltimer_ns() + 500;
+            else t_poll = globaltimer_ns() + 200;
         }
         if (progress) {
             t_stall = 0;
