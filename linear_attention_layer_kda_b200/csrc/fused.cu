@@ -6,27 +6,30 @@
 //
 //  * One CTA per SM, 16 warps, cooperative launch (all CTAs co-resident).
 //  * Projection pipeline (warps 0-7).  Every projection is a stream of 128 x 128 FP8 E4M3
-//    weight tiles (one fp32 block scale each).  Warp 0 loads tiles with TMA into an
-//    S-stage shared-memory ring; warp 1 loads the matching activation slice; warp 2 issues
-//    tcgen05.mma kind::f8f6f4 (M=128 weight rows, N = planes x padded batch, K=128 in four
-//    K=32 steps) into a double-buffered TMEM accumulator; warps 4-7 read TMEM, apply
+//    weight tiles (one fp32 block scale each).  Warp 0 lane 0 loads tiles with TMA into an
+//    S-stage shared-memory ring, each followed by the matching activation slice; warp 2 lane
+//    0 issues tcgen05.mma kind::f8f6f4 (M=128 weight rows, N = planes x padded batch, K=128
+//    in four K=32 steps) into one of eight TMEM accumulators; warps 4-7 read TMEM, apply
 //    weight scale x activation scale to the 128-wide K-block partial and accumulate in
-//    registers.  A CTA's run of tiles in one row block ends in a partial sum; the last of
-//    the row block's contributors adds the partials in a fixed order (deterministic).
+//    registers.  A CTA's run of tiles in one row block ends in a partial sum, published with
+//    a release increment of the row block's counter; the consumers (state units for q, k, v;
+//    the output reduction for W_o) add a row block's partials in slot order (deterministic).
 //  * Activations enter the tensor cores as FP8 "planes": a K-block of 128 values v with a
 //    power-of-two scale s is split v/s = p0 + p1 (+ p2 + p3) with every p an E4M3 value
 //    (each plane is the round-to-nearest residual of the previous ones).  Two planes hold
 //    a bf16 x exactly (up to the E4M3 subnormal floor, 2^-10 of the scale), four hold the
 //    fp32 readout o to about 2^-16 of its block maximum.  Products of E4M3 values are
 //    exact and accumulate in fp32, so no weight is ever dequantised in registers.
-//  * Vector warps (8-15): split x into planes, compute the beta and alpha-down gate rows
-//    (bf16, CUDA cores), then claim (sequence, o K-block) state units in head order: load
-//    the unit's fp32 state, wait until its heads' q/k/v are final, apply the gated delta
-//    rule in registers, write the state back in place, split o into planes and release
-//    the K-block to the output projection.
+//  * Vector warps (8-15): split x into planes (a share per CTA), compute the beta and
+//    alpha-down gate rows (bf16, CUDA cores), then run (sequence, o K-block) state units,
+//    assigned statically in head order: load the unit's fp32 state, wait until its heads'
+//    q/k/v are final, apply the gated delta rule in registers, split o into planes and
+//    release the K-block to the output projection, write the state back in place; the next
+//    unit's gates are computed while the current one waits.  Last, they add the W_o
+//    partials of their output rows into out.
 //  * Order: the q/k/v tiles of head group 0, 1, ..., then the W_o tiles of head group
-//    0, 1, ...  Heads become final group by group, so state traffic and the output
-//    projection overlap the weight stream instead of following it.
+//    0, 1, ...  The weight stream holds after its first tiles until x is split (bounded),
+//    so the x loads are not queued behind every SM's ring fill.
 //  * Every wait is bounded (global timer); on expiry the kernel records
 //    KDA_ERR_DEVICE_TIMEOUT, raises an abort flag every CTA polls, waits for its own
 //    copies and MMAs in flight, frees TMEM and returns.
