@@ -380,7 +380,7 @@ def main(argv=None):
     ap.add_argument("--clock-window", type=float, default=1.0,
                     help="seconds of untimed steps while nvidia-smi samples clocks before the timed region")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the host-buffer end-to-end loop")
-    ap.add_argument("--outdir", default=os.path.join(ROOT, "gpurun_out"))
+    ap.add_argument("--outdir", default=os.path.join(ROOT, "bench_out"), help="where the clock samples go")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     os.makedirs(args.outdir, exist_ok=True)
