@@ -250,7 +250,9 @@ KDA_API int kda_decode_abi_version(void);
  * All calls on one device share the one array: two calls that can run at the
  * same time (on different streams, or from host threads without ordering)
  * race on it and corrupt each other's activations.  Order them (one stream,
- * or events).  The set-up itself is thread-safe.
+ * or events).  The set-up itself is thread-safe.  The cached address belongs to
+ * the device context of the set-up: after cudaDeviceReset on that device it is
+ * stale and this entry point must not be called again in the process.
  */
 #define KDA_NOALLOC_MAX_SCRATCH_BYTES (1u << 20)
 KDA_API int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weights *w, float *state_inout,

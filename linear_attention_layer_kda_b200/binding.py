@@ -242,18 +242,31 @@ class KdaDecoder:
         for n, a in (("x", x), ("state", state), ("out", out)):
             if not a.is_cuda or not a.is_contiguous():
                 raise ValueError(f"{n} must be a contiguous CUDA tensor")
+        rows = batch * tokens
+        if x.shape[0] < rows or out.shape[0] < rows or state.shape[0] < batch:
+            raise ValueError(f"x and out need {rows} rows and state {batch} sequences")
         self._bind_stream()
         kda_decode_step_tokens(self.h, x.data_ptr(), weights, state.data_ptr(), out.data_ptr(), batch, tokens)
 
+    def _state_range(self, state, host, seq0: int, nseq: Optional[int]) -> int:
+        n = state.shape[0] - seq0 if nseq is None else nseq
+        c = self.cfg
+        need = n * c.num_heads * c.head_dk * c.head_dv * 4
+        if not state.is_cuda or not state.is_contiguous() or seq0 < 0 or n < 1 or seq0 + n > state.shape[0]:
+            raise ValueError("state must be a contiguous CUDA tensor holding sequences [seq0, seq0 + nseq)")
+        if host.is_cuda or not host.is_contiguous() or host.numel() * host.element_size() < need:
+            raise ValueError(f"host must be a contiguous host tensor of at least {need} bytes")
+        return n
+
     def checkpoint(self, state, host, seq0: int = 0, nseq: Optional[int] = None) -> None:
         """Enqueues a copy of sequences [seq0, seq0 + nseq) of `state` into the host tensor `host`."""
-        n = state.shape[0] - seq0 if nseq is None else nseq
+        n = self._state_range(state, host, seq0, nseq)
         self._bind_stream()
         kda_state_checkpoint(self.h, state.data_ptr(), seq0, n, host.data_ptr())
 
     def restore(self, host, state, seq0: int = 0, nseq: Optional[int] = None) -> None:
         """Enqueues a copy of the host tensor `host` into sequences [seq0, seq0 + nseq) of `state`."""
-        n = state.shape[0] - seq0 if nseq is None else nseq
+        n = self._state_range(state, host, seq0, nseq)
         self._bind_stream()
         kda_state_restore(self.h, host.data_ptr(), state.data_ptr(), seq0, n)
 
