@@ -113,3 +113,18 @@ def test_missing_library_raises(tmp_path):
             b.load(str(tmp_path / "nope.so"))
     finally:
         b._lib = saved
+
+
+def test_binding_rejects_bad_state_copies_without_a_device():
+    """The Python checks run before any library call (the decoder here has no handle)."""
+    import torch
+    from linear_attention_layer_kda_b200 import binding as b
+    dec = object.__new__(b.KdaDecoder)
+    dec.cfg = b.make_config(256, 2, 64, 64, 64, 4)
+    dec.h = None
+    per_seq = 2 * 64 * 64
+    host = torch.empty(4, per_seq)
+    with pytest.raises(ValueError, match="contiguous CUDA tensor"):
+        dec.checkpoint(torch.empty(4, 2, 64, 64), host)  # state not on a device
+    with pytest.raises(ValueError):
+        dec._state_range(torch.empty(4, 2, 64, 64), torch.empty(1), 0, 1)
