@@ -359,7 +359,7 @@ def kernel_rev() -> str:
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_attention_layer_kda_b200", "csrc")
-    for n in ("common.cuh", "sm100.cuh", "fused.cuh", "fused.cu", "simple.cu"):  # the engines' kernels
+    for n in ("common.cuh", "sm100.cuh", "fused.cuh", "fused.cu", "schedule.cu", "simple.cu"):  # the engines
         for line in open(os.path.join(d, n)):
             code = line.split("//", 1)[0].strip()  # comments and layout do not change the kernel
             if code:
