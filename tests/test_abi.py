@@ -128,3 +128,16 @@ def test_binding_rejects_bad_state_copies_without_a_device():
         dec.checkpoint(torch.empty(4, 2, 64, 64), host)  # state not on a device
     with pytest.raises(ValueError):
         dec._state_range(torch.empty(4, 2, 64, 64), torch.empty(1), 0, 1)
+
+
+def test_header_compiles_as_c99_and_host_calls_behave(lib, tmp_path):
+    """A plain C program against include/kda_decode.h and the built library."""
+    import subprocess
+    from linear_attention_layer_kda_b200 import binding
+    exe = str(tmp_path / "abi_check")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-o", exe, os.path.join(ROOT, "tests", "abi_check.c"),
+                           "-I" + os.path.join(ROOT, "include"), binding.LIB_PATH,
+                           "-Wl,-rpath," + os.path.dirname(binding.LIB_PATH)])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "abi_check ok" in r.stdout
