@@ -79,11 +79,11 @@ enum TraceSlot {
 // counters (uint32, monotonic across steps; targets are multiples of the step count)
 //   C_XQ          x K-blocks split into planes (B per K block per step)
 //   C_GATE        gate rows finished
-//   C_CLAIM0/1    (unused: state units are assigned statically)
+//   (words 2 and 3 are unused)
 //   C_ABORT       set by any wait that gives up
 //   off_oready+kb state units done for o K-block kb (B per step)
 //   off_rb+key    segments published for row block key (q, k, v, o row blocks)
-constexpr int C_XQ = 0, C_GATE = 1, C_CLAIM0 = 2, C_ABORT = 4, C_FIXED = 16;
+constexpr int C_XQ = 0, C_GATE = 1, C_ABORT = 4, C_FIXED = 16;
 
 struct __align__(16) VecSmem {
     float q[256], k[256];          // per head of the unit: q, k^  (heads_per_unit * dk)
