@@ -181,6 +181,14 @@ def test_invariant_beta1_unit_key_stores_value(literal):
     v = dbg["v"].reshape(shape.num_heads, shape.head_dv)
     Stk = np.einsum("hij,hi->hj", S1[0], kh)
     assert np.allclose(Stk, v, rtol=0, atol=1e-13 * np.abs(v).max())
+    # the readout contracts the UPDATED state with q: o = S'^T q.  A readout taken before the
+    # update (o = S^T q) differs from it by beta (v - S~^T k^)(k^ . q), which is large here.
+    q = dbg["q"].reshape(shape.num_heads, shape.head_dk)
+    o = dbg["o"][0].reshape(shape.num_heads, shape.head_dv)
+    after = np.einsum("hij,hi->hj", S1[0], q)
+    before = np.einsum("hij,hi->hj", inp.state0[0].astype(np.float64), q)
+    assert np.allclose(o, after, rtol=0, atol=1e-13 * np.abs(after).max())
+    assert np.abs(o - before).max() > 1e-3 * np.abs(after).max()
 
 
 @pytest.mark.parametrize("literal", [False, True])
@@ -196,6 +204,15 @@ def test_invariant_alpha0_forgets_state(literal):
     v = dbg["v"].reshape(shape.num_heads, shape.head_dv)
     want = beta[:, None, None] * kh[:, :, None] * v[:, None, :]
     assert np.allclose(S1[0], want, rtol=1e-14, atol=1e-300)
+    # with the old state forgotten, the readout after the update is o_h = beta_h v_h (k^_h . q_h)
+    # in closed form; a readout before the update would give S_0^T q instead
+    q = dbg["q"].reshape(shape.num_heads, shape.head_dk)
+    o = dbg["o"][0].reshape(shape.num_heads, shape.head_dv)
+    kq = np.einsum("hi,hi->h", kh, q)
+    want_o = beta[:, None] * v * kq[:, None]
+    assert np.allclose(o, want_o, rtol=0, atol=1e-13 * np.abs(want_o).max())
+    before = np.einsum("hij,hi->hj", inp.state0[0].astype(np.float64), q)
+    assert np.abs(o - before).max() > 1e-3 * np.abs(want_o).max()
 
 
 def test_invariant_idempotent_repeat():
