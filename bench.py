@@ -3,6 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload b8|b1|b12|b64]
 
+With --gpus N > 1 and no torchrun environment, the script starts N ranks of
+itself under torch.distributed.run (one process per GPU) and returns their
+exit status.
+
 A step is one kda_decode_step: one token for every sequence of the batch
 through projections, gates, the in-place state update, readout and output
 projection.  The default workload is batch 8, hidden 4096, 32 heads of
@@ -11,10 +15,12 @@ sequences, no collective on the data path); ``value`` is the whole-job
 decode steps/s, the max step time over ranks.
 
 Timing: W warm-up steps, then exactly K steps between CUDA events on the
-library's stream, bracketed by a barrier and a device synchronize.  Steps
+library's stream, bracketed by a barrier and a device synchronize; an event
+after every step gives the median, p10 and p90 of the per-step times.  Steps
 rotate over enough copies of weights + state (+ x, out) to exceed twice the
 L2 size, so every step streams from HBM, including the write-back of the
-previous step's state.
+previous step's state.  SM clocks and clock-event reasons are sampled through
+NVML while the timed steps run.
 """
 from __future__ import annotations
 
@@ -24,8 +30,10 @@ import json
 import math
 import os
 import statistics
+import socket
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -69,105 +77,182 @@ def measured_peaks() -> dict:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while it runs."""
+    """NVML sampling of the SM clock, power and clock-event reasons of one GPU.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    A background thread samples about every `period` seconds; `mark()` takes one
+    sample at once (called right after the timed steps are enqueued, while the GPU
+    runs them).  `stop(t0, t1)` reports the samples taken inside [t0, t1], the
+    host-clock span of the timed region; if none fell inside (a timed region far
+    shorter than the period), the marked sample and the samples next to the
+    window stand for it and `in_window` says so."""
 
-    def __init__(self, gpu_id: str, path: str):
-        self.path = path
-        self.proc = None
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_uuid: str, period: float = 0.002):
+        self.samples = []  # (host time, sm MHz, max sm MHz, power W, reasons mask)
+        self.err = None
+        self.period = period
+        self._stop = threading.Event()
+        self._lock = threading.Lock()
         try:
-            self.f = open(path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            u = device_uuid if device_uuid.startswith("GPU-") else "GPU-" + device_uuid
+            self.h = nv.nvmlDeviceGetHandleByUUID(u)
+            self.nv = nv
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM))
+        except Exception as e:  # noqa: BLE001 - no NVML: report why, time anyway
+            self.nv = None
+            self.err = f"nvml unavailable: {e}"
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
-    def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        self.proc.terminate()
+    def _sample(self):
+        nv = self.nv
+        t = time.perf_counter()
+        sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        sm, smax, reasons, n = [], [], set(), 0
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in open(self.path):
-            c = [x.strip() for x in ln.split(",")]
-            if len(c) < 9:
-                continue
+            pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        except Exception:  # noqa: BLE001
+            pw = None
+        rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        with self._lock:
+            self.samples.append((t, sm, self.max_mhz, pw, rs))
+
+    def _run(self):
+        while not self._stop.is_set():
             try:
-                sm.append(float(c[1]))
-                smax.append(float(c[2]))
-            except ValueError:
-                continue
-            n += 1
-            for nm, v in zip(names, c[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": n}
+                self._sample()
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(self.period)
+
+    def mark(self):
+        if self.nv is not None:
+            try:
+                self._sample()
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err], "samples": 0, "in_window": 0}
+        self._stop.set()
+        self.thread.join(timeout=5)
+        with self._lock:
+            allv = sorted(self.samples)
+        inside = [v for v in allv if t0 <= v[0] <= t1]
+        use = inside
+        if not use:  # nearest samples on both sides of a very short window
+            before = [v for v in allv if v[0] < t0][-1:]
+            after = [v for v in allv if v[0] > t1][:1]
+            use = before + after
+        reasons = set()
+        for v in use:
+            for name, attr in self.REASONS:
+                if v[4] & int(getattr(self.nv, attr, 0)):
+                    reasons.add(name)
+        pw = [v[3] for v in use if v[3] is not None]
+        return {"sm_mhz": statistics.median(v[1] for v in use) if use else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "power_w_max": max(pw) if pw else None, "samples": len(use), "in_window": len(inside),
+                "source": "nvml, sampled while the timed steps ran"}
 
 
-def gpu_id_for(local_rank: int) -> str:
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if vis:
-        ids = [v.strip() for v in vis.split(",") if v.strip()]
-        if local_rank < len(ids):
-            return ids[local_rank]
-    return str(local_rank)
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.lower().startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
 
-def oracle_rate(shape: I.KdaShape, inp, seqs: int, budget_s: float, max_steps: int):
-    """Oracle decode steps over `seqs` sequences; returns (full-batch steps/s, steps run, cores)."""
+def oracle_rate(shape: I.KdaShape, inp, seqs: int, budget_s: float, max_steps: int, threads: int = 0):
+    """Oracle decode steps over `seqs` sequences; returns (full-batch steps/s, steps run, threads used).
+
+    threads = 0 keeps OpenMP's default (every host core)."""
     import oracle
+    if threads:
+        oracle.set_num_threads(threads)
     m = oracle.OracleModel(inp, batch=seqs)
     S = inp.state0[:seqs].astype(np.float64).copy()
     n, t0 = 0, time.perf_counter()
-    while n < max_steps:
-        m.step(inp.x[0][:seqs], S)
-        n += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    m.close()
-    return (n * seqs / shape.batch) / dt, n, oracle.num_threads()
+    try:
+        while n < max_steps:
+            m.step(inp.x[n % len(inp.x)][:seqs], S)
+            n += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        used = oracle.num_threads()
+    finally:
+        m.close()
+        if threads:
+            oracle.set_num_threads(os.cpu_count() or 1)
+    return (n * seqs / shape.batch) / dt, n, used
 
 
-def run_reference(args, shape, rank):
-    """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+L2_ASSUMED = 126 * 2 ** 20  # B200 L2; the GPU arm uses the device's own figure if it is larger
+
+
+def rotation_sets(shape: I.KdaShape, l2: int = L2_ASSUMED) -> int:
+    """Copies of (weights, state, x, out) the steps rotate over so that the set exceeds twice L2."""
+    return max(2, math.ceil(2 * l2 / ideal_bytes(shape, shape.batch)))
+
+
+def workload_config(shape, n, sets):
+    """The workload as both arms report it (identical dictionaries for the same shape and N)."""
+    steps_note = (f"{shape.steps} sequential decode steps, fresh x each step, state carried in place"
+                  if shape.steps > 1 else "one decode step per timed iteration")
+    return {"workload": shape.name, "batch_per_gpu": shape.batch, "global_batch": shape.batch * n,
+            "hidden": shape.hidden, "num_heads": shape.num_heads, "head_dk": shape.head_dk,
+            "head_dv": shape.head_dv, "alpha_rank": shape.alpha_rank,
+            "weights": "FP8 E4M3 q/k/v/o with fp32 128x128 block scales; bf16 alpha (low rank) and beta",
+            "state": "fp32 [B, nh, dk, dv], updated in place", "out": "fp32", "steps": steps_note,
+            "parallelism": f"dp{n} (independent sequences per GPU, weights replicated, no collective)",
+            "l2": f"inputs larger than L2: steps rotate over {sets} copies of weights + state "
+                  f"({ideal_bytes(shape, shape.batch) / 1e6:.1f} MB each, > 2x the L2)"}
+
+
+def run_reference(args, shape, rank, world):
+    """Reference arm: the fp64 oracle on the host cores (rank 0 only; other ranks exit at once)."""
     if rank != 0:
         return 0
     import oracle
     oracle.build()
-    inp = I.generate(shape.replace(steps=1))
+    steps = max(1, shape.steps)
+    inp = I.generate(shape.replace(steps=steps))
     seqs = shape.batch if args.steps <= 50 else 1
     m = oracle.OracleModel(inp, batch=seqs)
     S = inp.state0[:seqs].astype(np.float64).copy()
-    for _ in range(args.warmup):
-        m.step(inp.x[0][:seqs], S)
+    for i in range(args.warmup):
+        m.step(inp.x[i % steps][:seqs], S)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        m.step(inp.x[0][:seqs], S)
+    for i in range(args.steps):
+        m.step(inp.x[i % steps][:seqs], S)
     dt = time.perf_counter() - t0
     m.close()
     full_steps_per_s = (args.steps * seqs / shape.batch) / dt
     sample = (f"each step: one fp64 oracle decode step over {seqs} of the {shape.batch} sequences "
               f"(rank-1 form, OpenMP), scaled to full-batch steps")
     line = {
-        "impl": "reference", "metric": METRIC, "value": full_steps_per_s, "unit": "steps/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": full_steps_per_s, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / full_steps_per_s,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(shape, args.gpus, "cpu"),
+        "config": workload_config(shape, world, rotation_sets(shape)),
         "cpu_baseline": {"value": full_steps_per_s, "unit": "steps/s", "cores": oracle.num_threads(),
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": full_steps_per_s, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -179,10 +264,12 @@ def rank_inputs(shape: I.KdaShape, rank: int, world: int):
     sequences, rows rank*B .. rank*B + B - 1 of the job's counter-based streams, so the N
     ranks together hold exactly the sequences of one batch of N*B (data parallel, no
     collective on the data path)."""
-    inp = I.generate(shape.replace(steps=1))
+    steps = max(1, shape.steps)
+    inp = I.generate(shape.replace(steps=steps))
     if world > 1:
         B = shape.batch
-        inp.x[0] = I.gen_x(shape, 0, batch=B, row0=rank * B)
+        for t in range(steps):
+            inp.x[t] = I.gen_x(shape, t, batch=B, row0=rank * B)
         inp.state0 = I.gen_state(shape, batch=B, row0=rank * B)
     return inp
 
@@ -203,14 +290,10 @@ def job_steps_per_s(ms_per_step_slowest: float, world: int) -> float:
     return world * 1000.0 / ms_per_step_slowest
 
 
-def workload_config(shape, n, l2_note):
-    return {"workload": shape.name, "batch_per_gpu": shape.batch, "global_batch": shape.batch * n,
-            "hidden": shape.hidden, "num_heads": shape.num_heads, "head_dk": shape.head_dk,
-            "head_dv": shape.head_dv, "alpha_rank": shape.alpha_rank,
-            "weights": "FP8 E4M3 q/k/v/o with fp32 128x128 block scales; bf16 alpha (low rank) and beta",
-            "state": "fp32 [B, nh, dk, dv], updated in place", "out": "fp32",
-            "parallelism": f"dp{n} (independent sequences per GPU, weights replicated, no collective)",
-            "l2": l2_note}
+def step_percentiles(step_ms):
+    """median, p10, p90 of per-step times (ms)."""
+    v = np.asarray(step_ms, dtype=np.float64)
+    return float(np.median(v)), float(np.percentile(v, 10)), float(np.percentile(v, 90))
 
 
 # ------------------------------------------------------------------ our arm
@@ -227,15 +310,16 @@ def run_ours(args, shape, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     B = shape.batch
     props = torch.cuda.get_device_properties(dev)
-    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    l2 = max(L2_ASSUMED, int(getattr(props, "L2_cache_size", L2_ASSUMED)))
 
     inp = rank_inputs(shape, rank, world)
+    T = len(inp.x)  # fresh x per step for multi-step workloads
     set_bytes = ideal_bytes(shape, B)
-    R = max(2, math.ceil(2 * l2 / set_bytes))
+    R = rotation_sets(shape, l2)
     wts = [tensors.to_device_weights(inp, dev) for _ in range(R)]
     ws = [tensors.weights_struct(w) for w in wts]
     states = [tensors.state_tensor(inp.state0, dev) for _ in range(R)]
-    xs = [tensors.bf16_tensor(inp.x[0], dev) for _ in range(R)]
+    xs = [tensors.bf16_tensor(inp.x[t], dev) for t in range(T)]
     outs = [torch.empty(B, shape.hidden, device=dev, dtype=torch.float32) for _ in range(R)]
     dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, B,
                              engine=args.engine)
@@ -244,16 +328,15 @@ def run_ours(args, shape, rank, world, local_rank):
 
     def one(i):
         j = i % R
-        dec.step(xs[j], ws[j], states[j], outs[j])
+        dec.step(xs[i % T], ws[j], states[j], outs[j])
 
     for i in range(max(3, args.warmup)):
         one(i)
     dec.sync()
     torch.cuda.synchronize()
 
-    clk = ClockSampler(gpu_id_for(local_rank), os.path.join(args.outdir, f"clocks_rank{rank}.csv")) \
-        if rank == 0 else None
-    # untimed load window so the clock sampler sees the step loop for about a second
+    clk = ClockSampler(str(getattr(props, "uuid", ""))) if rank == 0 else None
+    # untimed load so the clocks settle under load before the timed region
     t_end = time.perf_counter() + (args.clock_window if clk else 0.0)
     i = 0
     while time.perf_counter() < t_end:
@@ -267,45 +350,54 @@ def run_ours(args, shape, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    h0 = time.perf_counter()
+    evs[0].record(stream)
     for i in range(args.steps):
         one(i)
-    ev1.record(stream)
+        evs[i + 1].record(stream)
+    if clk:
+        clk.mark()  # the GPU is still running the steps just enqueued
     torch.cuda.synchronize()
+    h1 = time.perf_counter()
     dec.sync()  # raises on a recorded device-side timeout
     if world > 1:
         dist.barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    clocks = clk.stop() if clk else None
+    ms_total = evs[0].elapsed_time(evs[-1])
+    step_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    clocks = clk.stop(h0, h1) if clk else None
 
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_per_step = ms_total / args.steps
     value = job_steps_per_s(ms_per_step, world)
+    med, p10, p90 = step_percentiles(step_ms)
 
     # end to end through the host-buffer entry point: H2D x, step, D2H out, sync, every step,
     # on every rank; the slowest rank's wall time sets the job's rate
-    xh = torch.from_numpy(inp.x[0].view(np.int16)).view(torch.bfloat16).pin_memory()
+    xh = [torch.from_numpy(inp.x[t].view(np.int16)).view(torch.bfloat16).pin_memory() for t in range(T)]
     oh = torch.empty(B, shape.hidden, dtype=torch.float32).pin_memory()
     n_e2e = args.e2e_steps if args.e2e_steps > 0 else max(10, min(args.steps, 2000))
     for i in range(3):
-        dec.step_host(xh, ws[i % R], states[i % R], oh)
+        dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
     if world > 1:
         dist.barrier()
     t0 = time.perf_counter()
     for i in range(n_e2e):
-        dec.step_host(xh, ws[i % R], states[i % R], oh)
+        dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
     dt = max_over_ranks(time.perf_counter() - t0, world, dev)
     e2e = {"value": job_steps_per_s(1000.0 * dt / n_e2e, world), "unit": "steps/s",
-           "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 4), "steps": n_e2e}
+           "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 4), "steps": n_e2e}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n, cores = oracle_rate(shape, inp, seqs=B, budget_s=args.cpu_seconds, max_steps=1000)
-        cpu = {"value": rate, "unit": "steps/s", "cores": cores, "kind": "oracle",
+        rate1, n1, _ = oracle_rate(shape, inp, seqs=1, budget_s=min(5.0, args.cpu_seconds), max_steps=50, threads=1)
+        cpu = {"value": rate, "unit": "steps/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                "sample": f"{n} fp64 oracle decode steps of the same workload (batch {B}, rank-1 form, "
-                         f"OpenMP), about {args.cpu_seconds:.0f} s of CPU work"}
+                         f"OpenMP on {cores} threads), about {args.cpu_seconds:.0f} s of CPU work",
+               "single_thread": {"value": rate1, "unit": "steps/s",
+                                 "sample": f"{n1} oracle steps of one sequence on 1 thread, scaled to "
+                                           f"full-batch steps"}}
 
     dec.close()
     if world > 1:
@@ -332,9 +424,10 @@ def run_ours(args, shape, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(shape, world, f"rotating {R} weight+state sets of {set_bytes / 1e6:.1f} MB "
-                                               f"(> 2x the {l2 / 2 ** 20:.0f} MiB L2)"),
+        "config": workload_config(shape, world, R),
         "tokens_per_s": value * B,
+        "step_us": {"median": med * 1e3, "p10": p10 * 1e3, "p90": p90 * 1e3,
+                    "note": "per-step CUDA events on the launching stream (rank 0)"},
         "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
         "engine": {1: "simple", 2: "fused"}.get(engine, str(engine)),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -359,7 +452,7 @@ def kernel_rev() -> str:
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_attention_layer_kda_b200", "csrc")
-    for n in ("common.cuh", "sm100.cuh", "fused.cuh", "fused.cu", "schedule.cu", "simple.cu"):  # the engines
+    for n in sorted(f for f in os.listdir(d) if f.endswith((".cu", ".cuh"))):  # the engines and the ABI
         for line in open(os.path.join(d, n)):
             code = line.split("//", 1)[0].strip()  # comments and layout do not change the kernel
             if code:
@@ -367,7 +460,22 @@ def kernel_rev() -> str:
     return h.hexdigest()[:16]
 
 
-def main(argv=None):
+# ------------------------------------------------------------------ launcher
+
+def free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_command(nproc: int, argv, port: int, limit_s: int):
+    """torch.distributed.run command that starts `nproc` ranks of this script (one per GPU)."""
+    return ["timeout", "-k", "60", str(limit_s), sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={nproc}", "--master-addr", "127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__)] + list(argv)
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -377,19 +485,33 @@ def main(argv=None):
     ap.add_argument("--engine", type=int, default=0, help="0 auto, 1 simple, 2 fused")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--clock-window", type=float, default=1.0,
-                    help="seconds of untimed steps while nvidia-smi samples clocks before the timed region")
+    ap.add_argument("--clock-window", type=float, default=0.5,
+                    help="seconds of untimed steps before the timed region, so clocks settle under load")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the host-buffer end-to-end loop")
-    ap.add_argument("--outdir", default=os.path.join(ROOT, "bench_out"), help="where the clock samples go")
-    args = ap.parse_args(argv)
+    ap.add_argument("--launch-limit", type=int, default=900, help="seconds before a self-launched job is killed")
+    ap.add_argument("--print-rank", action="store_true", help=argparse.SUPPRESS)  # launcher self-check
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
+    args = parse_args(argv)
     args.warmup = max(3, args.warmup)
-    os.makedirs(args.outdir, exist_ok=True)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # not under torchrun: start one rank per GPU and hand back their exit status
+        return subprocess.call(launch_command(args.gpus, argv, free_port(), args.launch_limit))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"bench.py: {world} ranks are running but --gpus is {args.gpus}; refusing to report", file=sys.stderr)
+        return 2
+    if args.print_rank:
+        print(json.dumps({"rank": rank, "world_size": world, "local_rank": local_rank}), flush=True)
+        return 0
     shape = I.CONFIGS[WORKLOADS[args.workload]]
     if args.impl == "reference":
-        return run_reference(args, shape, rank)
+        return run_reference(args, shape, rank, world)
     return run_ours(args, shape, rank, world, local_rank)
 
 

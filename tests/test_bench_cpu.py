@@ -39,3 +39,43 @@ def test_kernel_revision_ignores_comments(tmp_path, monkeypatch):
     with open(fake / "fused.cu", "a") as f:
         f.write("static int kda_extra_symbol_for_the_test = 1;\n")
     assert bench.kernel_rev() != rev
+
+
+def test_step_percentiles():
+    med, p10, p90 = bench.step_percentiles([float(i) for i in range(1, 102)])
+    assert med == 51.0 and p10 == 11.0 and p90 == 91.0
+
+
+def test_launcher_starts_one_rank_per_gpu():
+    """`--gpus 2` without a torchrun environment starts two ranks of bench.py with RANK and
+    WORLD_SIZE set (checked with the launcher self-check flag, which exits before any CUDA)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2", "--print-rank",
+                        "--launch-limit", "120"], env=env, capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert sorted(d["rank"] for d in lines) == [0, 1]
+    assert all(d["world_size"] == 2 for d in lines)
+
+
+def test_refuses_a_line_for_a_different_gpu_count(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--gpus", "2", "--print-rank"]) == 2
+    assert "refusing" in capsys.readouterr().err
+
+
+def test_reference_arm_reports_the_same_config_as_ours(capsys):
+    """The reference arm's config equals the dictionary the GPU arm prints for the same workload."""
+    import json
+    shape = I.CONFIGS[0]
+    args = bench.parse_args(["--steps", "2", "--warmup", "0"])
+    assert bench.run_reference(args, shape, 0, 1) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 1
+    assert line["config"] == bench.workload_config(shape, 1, bench.rotation_sets(shape))
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["cpu_model"]
