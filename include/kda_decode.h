@@ -35,7 +35,15 @@
  *     the host (null or misaligned pointers, sizes) are returned before
  *     anything is enqueued.  A device-side bounded wait that gives up sets a
  *     status word that the next kda_decode_step / kda_decode_sync returns as
- *     KDA_ERR_DEVICE_TIMEOUT.
+ *     KDA_ERR_DEVICE_TIMEOUT.  Steps enqueued after the one that timed out,
+ *     before the error was returned, stop without doing their work: after
+ *     KDA_ERR_DEVICE_TIMEOUT treat every step enqueued since the last
+ *     successful kda_decode_sync as not run (outputs and state unwritten).
+ *     If an aborted kernel also could not drain its own copies in flight, the
+ *     handle is unusable: every later call on it returns
+ *     KDA_ERR_DEVICE_TIMEOUT; destroy it and create a new one.
+ *   - The handle belongs to the device that was current at kda_decode_init;
+ *     that device must be current whenever the handle enqueues work.
  *   - There is no CPU fallback: without a usable sm_100 device every call
  *     fails with KDA_ERR_NO_DEVICE or KDA_ERR_CUDA.
  *   - A handle is not thread-safe; use one handle per stream.
@@ -178,6 +186,19 @@ KDA_API int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weight
 KDA_API int kda_state_checkpoint(kda_handle h, const float *state, int seq0, int nseq, void *host_dst);
 KDA_API int kda_state_restore(kda_handle h, const void *host_src, float *state, int seq0, int nseq);
 
+/*
+ * Launch overlap between consecutive steps (on by default).  A fused-engine step is
+ * launched with programmatic stream serialization: its kernel may start on the SMs the
+ * kernel enqueued just before it frees, and there, before that kernel has finished, it
+ * already streams the first weight tiles of the step into shared memory.  It touches x,
+ * the state and its scratch only after the preceding kernel has completed, so only the
+ * weights are read early: a kernel that WRITES a step's weights must not be enqueued on the
+ * stream immediately before that step while the overlap is on.  on = 0 restores strict
+ * stream order (the step then also uses a cooperative launch, which makes the runtime check
+ * that every CTA of the step can be resident at once).  Applies to later steps.
+ */
+KDA_API int kda_decode_set_launch_overlap(kda_handle h, int on);
+
 /* Waits for the handle's stream; returns the device status of the steps since
  * the last check (KDA_OK or KDA_ERR_DEVICE_TIMEOUT) and clears it. */
 KDA_API int kda_decode_sync(kda_handle h);
@@ -237,22 +258,25 @@ KDA_API int kda_decode_abi_version(void);
  * and nothing is cleared.
  *
  *   cfg          shape and out dtype as for kda_decode_init (validated the
- *                same way; max_batch and engine are not used)
+ *                same way; max_batch and engine are ignored, not checked)
  *   x, w, state_inout, out   as for kda_decode_step (device memory)
  *   batch        1 .. any, within the scratch limit above
  *   cuda_stream  cudaStream_t passed as void* (NULL = legacy default stream)
  *
- * Set-up: the first call on each device, with that device current, looks up
- * the array's device address (cudaGetSymbolAddress, which may also load the
- * library's device code on that device) and caches it; later calls only
- * read the cache.  Make that first call before any stream capture begins.
+ * Set-up: the first call in each CUDA context (normally a device's primary
+ * context, bound with cudaSetDevice), with that context current, looks up the
+ * array's device address (cudaGetSymbolAddress, which may also load the
+ * library's device code on that device) and caches it under the context;
+ * later calls only read the cache.  Make that first call before any stream
+ * capture begins.
  *
  * All calls on one device share the one array: two calls that can run at the
  * same time (on different streams, or from host threads without ordering)
  * race on it and corrupt each other's activations.  Order them (one stream,
  * or events).  The set-up itself is thread-safe.  The cached address belongs to
- * the device context of the set-up: after cudaDeviceReset on that device it is
- * stale and this entry point must not be called again in the process.
+ * the context of the set-up: once that context is destroyed (cudaDeviceReset,
+ * cuCtxDestroy) the entry is stale, and this entry point must not be called
+ * again in the process.
  */
 #define KDA_NOALLOC_MAX_SCRATCH_BYTES (1u << 20)
 KDA_API int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weights *w, float *state_inout,

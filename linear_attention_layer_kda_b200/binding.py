@@ -34,6 +34,7 @@ EXPORTS = (
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
     "kda_decode_step_noalloc", "kda_decode_step_tokens", "kda_state_checkpoint", "kda_state_restore",
+    "kda_decode_set_launch_overlap",
 )
 KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
 KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
@@ -94,6 +95,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_decode_step_tokens": (I, [P, P, ctypes.POINTER(kda_weights), P, P, I, I]),
         "kda_state_checkpoint": (I, [P, P, I, I, P]),
         "kda_state_restore": (I, [P, P, P, I, I]),
+        "kda_decode_set_launch_overlap": (I, [P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -138,6 +140,10 @@ def kda_state_restore(h: int, host_src: int, state: int, seq0: int, nseq: int) -
 
 def kda_decode_step_host(h: int, x_host: int, w: kda_weights, state: int, out_host: int, batch: int) -> None:
     _check(load().kda_decode_step_host(h, x_host, ctypes.byref(w), state, out_host, batch), "kda_decode_step_host", h)
+
+
+def kda_decode_set_launch_overlap(h: int, on: bool) -> None:
+    _check(load().kda_decode_set_launch_overlap(h, 1 if on else 0), "kda_decode_set_launch_overlap", h)
 
 
 def kda_decode_sync(h: int) -> None:
@@ -272,6 +278,10 @@ class KdaDecoder:
 
     def sync(self) -> None:
         kda_decode_sync(self.h)
+
+    def set_launch_overlap(self, on: bool) -> None:
+        """Overlap of consecutive fused steps (programmatic dependent launch); on by default."""
+        kda_decode_set_launch_overlap(self.h, on)
 
     def debug_tensor(self, which: int, batch: int):
         """fp32 copy of one intermediate of the last step (KDA_DEBUG_*), shape [batch, n]."""

@@ -2,12 +2,14 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <map>
 #include <mutex>
 #include <new>
 #include <string>
 
 #include "common.cuh"
 #include "fused.cuh"
+#include "status.h"
 
 struct kda_handle_s {
     kda_config cfg{};
@@ -22,6 +24,7 @@ struct kda_handle_s {
     void *x_stage = nullptr;    // device staging of x for kda_decode_step_host
     void *out_stage = nullptr;  // device staging of out for kda_decode_step_host
     kda::FusedState fused;
+    bool fatal = false;  // a kernel gave up draining its copies after an abort: never step again
     std::string last_error;
 };
 
@@ -133,18 +136,22 @@ int check_step(kda_handle h, const void *x, const kda_weights *w, const float *s
     return KDA_OK;
 }
 
-// Reads and clears the mapped status word (call after the stream is idle, or to peek).
+// Reads and clears the mapped status words (after the stream is idle, or to peek).  After a
+// timeout the counters of the aborted step are inconsistent, so the next step resets them.
 int take_device_status(kda_handle h)
 {
-    volatile int *sp = h->status_host;
-    const int st = sp[0], where = sp[1];
+    std::string msg;
+    const int st = kda::take_status(h->status_host, &h->fatal, &msg);
     if (st == KDA_OK) return KDA_OK;
-    sp[0] = KDA_OK;
-    sp[1] = 0;
-    h->fused.needs_reset = true;  // flags and counters of the aborted step are inconsistent
-    if (st == KDA_ERR_DEVICE_TIMEOUT)
-        return fail(h, st, "a device-side bounded wait expired (wait site " + std::to_string(where) + ")");
-    return fail(h, st, "device reported an error");
+    h->fused.needs_reset = true;
+    return fail(h, st, msg);
+}
+
+// A handle whose kernel could not drain its own copies after an abort is never used again.
+int check_usable(kda_handle h)
+{
+    if (!h->fatal) return KDA_OK;
+    return fail(h, KDA_ERR_DEVICE_TIMEOUT, "handle unusable: an aborted step did not drain its copies in flight");
 }
 
 int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state, void *out, int batch)
@@ -165,9 +172,38 @@ int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state
 // fixed array per device, for callers that may not allocate (see the header).
 __device__ __align__(256) unsigned char g_noalloc_scratch[KDA_NOALLOC_MAX_SCRATCH_BYTES];
 
-constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[kNoAllocMaxDevices];  // device address of the array, per device (set-up cache)
+std::map<void *, void *> g_noalloc_ptr;  // device address of the array, per CUDA context (set-up cache)
+
+typedef CUresult (*PFN_ctxGetCurrent)(CUcontext *);
+
+// The CUDA context current on this thread (the runtime binds the device's primary context on
+// first use; cudaSetDevice does that without allocating), or null.
+CUcontext current_context(int dev)
+{
+    static PFN_ctxGetCurrent fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_ctxGetCurrent>(p);
+        else
+            (void)cudaGetLastError();
+    });
+    if (!fn) return nullptr;
+    CUcontext ctx = nullptr;
+    if (fn(&ctx) != CUDA_SUCCESS) return nullptr;
+    if (!ctx) {
+        if (cudaSetDevice(dev) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        if (fn(&ctx) != CUDA_SUCCESS) return nullptr;
+    }
+    return ctx;
+}
 
 // Activations of `batch` sequences inside the array (same order as a handle's scratch);
 // returns false if they do not fit.
@@ -193,8 +229,13 @@ extern "C" {
 int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weights *w, float *state_inout,
                             void *out, int batch, void *cuda_stream)
 {
+    if (!cfg) return KDA_ERR_INVALID_ARG;
+    // only the shape and out dtype matter here: max_batch and engine are not used
+    kda_config shape = *cfg;
+    shape.max_batch = 1;
+    shape.engine = KDA_ENGINE_AUTO;
     std::string why;
-    int rc = validate_config(cfg, &why);
+    int rc = validate_config(&shape, &why);
     if (rc) return rc;
     if (batch < 1) return KDA_ERR_INVALID_ARG;
     if (!x || !state_inout || !out) return KDA_ERR_INVALID_ARG;
@@ -210,11 +251,13 @@ int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weig
 
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return KDA_ERR_NO_DEVICE; }
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return KDA_ERR_NO_DEVICE;
+    CUcontext ctx = current_context(dev);
+    if (!ctx) return KDA_ERR_NO_DEVICE;
     void *base = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {  // set-up, once per device, with that device current
+        auto it = g_noalloc_ptr.find(ctx);
+        if (it == g_noalloc_ptr.end()) {  // set-up, once per context, with its device current
             int major = 0;
             if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
                 (void)cudaGetLastError();
@@ -226,9 +269,9 @@ int kda_decode_step_noalloc(const kda_config *cfg, const void *x, const kda_weig
                 (void)cudaGetLastError();
                 return KDA_ERR_CUDA;
             }
-            g_noalloc_ptr[dev] = p;
+            it = g_noalloc_ptr.emplace(ctx, p).first;
         }
-        base = g_noalloc_ptr[dev];
+        base = it->second;
     }
     noalloc_layout(*cfg, batch, static_cast<char *>(base), &s);
     const kda::Dims d = dims_of(*cfg, batch);
@@ -327,6 +370,7 @@ int kda_decode_init(const kda_config *cfg, kda_handle *out_handle)
     if (e == cudaSuccess) {
         h->status_host[0] = KDA_OK;
         h->status_host[1] = 0;
+        h->status_host[2] = 0;
         e = cudaHostGetDevicePointer((void **)&h->status, h->status_host, 0);
     }
     if (e == cudaSuccess) e = kda::fused_init(dims_of(*cfg, cfg->max_batch), &h->fused);
@@ -349,6 +393,13 @@ int kda_decode_set_stream(kda_handle h, void *stream)
     return KDA_OK;
 }
 
+int kda_decode_set_launch_overlap(kda_handle h, int on)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    h->fused.overlap = on != 0;
+    return KDA_OK;
+}
+
 int kda_decode_engine(kda_handle h, int batch)
 {
     if (!h || batch < 1 || batch > h->cfg.max_batch) return -KDA_ERR_INVALID_ARG;
@@ -365,7 +416,9 @@ int kda_decode_launches_per_step(kda_handle h, int batch)
 int kda_decode_step(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out, int batch)
 {
     if (!h) return KDA_ERR_INVALID_ARG;
-    int rc = check_step(h, x, w, state_inout, out, batch);
+    int rc = check_usable(h);
+    if (rc) return rc;
+    rc = check_step(h, x, w, state_inout, out, batch);
     if (rc) return rc;
     // A timeout recorded by an earlier step is reported (and cleared) here.
     rc = take_device_status(h);
@@ -378,7 +431,9 @@ int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w,
 {
     if (!h) return KDA_ERR_INVALID_ARG;
     if (!x_host || !out_host) return fail(h, KDA_ERR_INVALID_ARG, "null host buffer");
-    int rc = check_step(h, h->x_stage, w, state_inout, h->out_stage, batch);
+    int rc = check_usable(h);
+    if (rc) return rc;
+    rc = check_step(h, h->x_stage, w, state_inout, h->out_stage, batch);
     if (rc) return rc;
     rc = take_device_status(h);
     if (rc) return rc;
@@ -399,6 +454,7 @@ int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, fl
 {
     if (!h) return KDA_ERR_INVALID_ARG;
     if (tokens < 1) return fail(h, KDA_ERR_INVALID_ARG, "tokens must be >= 1");
+    if (int rc0 = check_usable(h)) return rc0;
     if (tokens == 1) return kda_decode_step(h, x, w, state_inout, out, batch);
     if (batch < 1 || (long long)batch * tokens > h->cfg.max_batch)
         return fail(h, KDA_ERR_INVALID_ARG, "batch * tokens must be in [1, max_batch]");
@@ -452,7 +508,8 @@ int kda_decode_sync(kda_handle h)
     if (!h) return KDA_ERR_INVALID_ARG;
     cudaError_t e = cudaStreamSynchronize(h->stream);
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
-    return take_device_status(h);
+    const int st = take_device_status(h);
+    return st ? st : check_usable(h);
 }
 
 int kda_decode_debug_copy(kda_handle h, int which, void *dst, size_t bytes)

@@ -5,15 +5,21 @@
 // split over every SM; Kiln's "one scale per kernel tile" for the FP8 weights):
 //
 //  * One CTA per SM, 16 warps, cooperative launch (all CTAs co-resident).
-//  * Projection pipeline (warps 0-7).  Every projection is a stream of 128 x 128 FP8 E4M3
-//    weight tiles (one fp32 block scale each).  Warp 0 lane 0 loads tiles with TMA into an
-//    S-stage shared-memory ring, each followed by the matching activation slice; warp 2 lane
-//    0 issues tcgen05.mma kind::f8f6f4 (M=128 weight rows, N = planes x padded batch, K=128
-//    in four K=32 steps) into one of eight TMEM accumulators; warps 4-7 read TMEM, apply
-//    weight scale x activation scale to the 128-wide K-block partial and accumulate in
-//    registers.  A CTA's run of tiles in one row block ends in a partial sum, published with
-//    a release increment of the row block's counter; the consumers (state units for q, k, v;
-//    the output reduction for W_o) add a row block's partials in slot order (deterministic).
+//  * Projection pipeline (warps 0-7).  Every projection is a stream of weight tiles of N
+//    rows (256 while the batch allows) x one 128-wide K block; each 128 x 128 sub-block has
+//    one fp32 scale.  Warp 0 lane 0 loads the weight tiles with TMA into a shared-memory
+//    ring, each followed by the activation tile of its K block (x planes, or o planes once
+//    the state units have released them).  Warp 2 lane 0 issues tcgen05.mma kind::f8f6f4 with the
+//    ACTIVATIONS as the M = 128 operand and the WEIGHTS as the N operand (K = 128 in four
+//    K = 32 steps) into one of two TMEM accumulators, and commits once per tile: a
+//    tcgen05.mma costs about the same whatever its N, so 256 weight rows per instruction and
+//    one commit per 32 KB keep the tensor pipe ahead of HBM.  Warps 4-7 (one per TMEM lane
+//    quarter) read the accumulator with 16x256b loads, which hand each thread both planes of
+//    one sequence, apply weight scale x activation scale per 128 x 128 block and keep
+//    running sums in registers; a CTA's run of tiles in one row group ends in a partial sum.
+//    Warp 3 lane 0 publishes it with a release increment of the row group's counter, so the
+//    fence that the release implies never holds up the epilogue; consumers add a row group's
+//    partials in slot order (deterministic).
 //  * Activations enter the tensor cores as FP8 "planes": a K-block of 128 values v with a
 //    power-of-two scale s is split v/s = p0 + p1 (+ p2 + p3) with every p an E4M3 value
 //    (each plane is the round-to-nearest residual of the previous ones).  Two planes hold
@@ -27,9 +33,12 @@
 //    release the K-block to the output projection, write the state back in place; the next
 //    unit's gates are computed while the current one waits.  Last, they add the W_o
 //    partials of their output rows into out.
-//  * Order: the q/k/v tiles of head group 0, 1, ..., then the W_o tiles of head group
-//    0, 1, ...  The weight stream holds after its first tiles until x is split (bounded),
-//    so the x loads are not queued behind every SM's ring fill.
+//  * Order: the weight tiles are dealt to the SMs in waves, earliest heads first (see
+//    schedule.cu), so early heads' state units and W_o tiles overlap the rest of the
+//    stream.  Few stages are kept in flight per SM: HBM is saturated with less, and every
+//    extra byte queued in the memory system delays the flags and partial sums the step's
+//    dependency chain runs on.  For the same reason the weight stream holds after its first
+//    tiles until x is split (bounded).
 //  * Every wait is bounded (global timer); on expiry the kernel records
 //    KDA_ERR_DEVICE_TIMEOUT, raises an abort flag every CTA polls, waits for its own
 //    copies and MMAs in flight, frees TMEM and returns.
@@ -39,6 +48,7 @@
 #include <algorithm>
 #include <map>
 #include <mutex>
+#include <utility>
 
 #include "fused.cuh"
 #include "sm100.cuh"
@@ -50,13 +60,15 @@ using namespace sm100;
 
 constexpr int kThreads = 512;
 constexpr int kMaxBP = 64;
-constexpr int kTileBytes = 128 * 128;
-constexpr int kMaxStages = 12;   // ring stages (weight tile + activation planes)
-constexpr int kMaxAcc = 8;       // TMEM accumulator buffers
+constexpr int kMaxStages = 8;    // ring stages (weight tile + activation tile)
+constexpr int kMaxAcc = 4;       // TMEM accumulator buffers
+constexpr int kEpiWarps = 4;     // warps 4-7, one per TMEM lane quarter
 constexpr int kMaxTilesPerCta = 512;
 constexpr int kTmemCols = 512;
-constexpr int kEarlyTiles = 2;                 // weight copies issued before x is known final
-constexpr uint64_t kEarlyHoldNs = 6000;        // longest hold of the rest of the stream
+constexpr int kMaxStagesDefault = 3;  // stages in flight unless KDA_STAGES says otherwise
+constexpr int kEarlyTilesDefault = 1;  // weight copies issued before x is known final (KDA_EARLY_TILES)
+constexpr uint64_t kEarlyHoldNs = 6000;  // longest hold of the rest of the stream
+constexpr int kSegBars = 32;          // segment hand-off barriers (epilogue -> publisher), reused mod 32
 
 // Optional timeline (compile with -DKDA_TRACE): per CTA, kTraceSlots global-timer stamps.
 #ifdef KDA_TRACE
@@ -71,7 +83,10 @@ constexpr uint64_t kEarlyHoldNs = 6000;        // longest hold of the rest of th
 #endif
 enum TraceSlot {
     TR_START = 0, TR_XREADY, TR_FIRST_MMA, TR_QKV_DONE, TR_EPI_DONE, TR_XQ_DONE, TR_GATES_DONE,
-    TR_UNIT0 = 7,  /* 3 stamps per unit: claimed, inputs ready, done; 4 units */
+    TR_UNIT0 = 7,  /* 3 stamps per unit: claimed, inputs ready, done; 2 units */
+    TR_UNIT_SUMS = 13, /* units 0, 1: partial sums loaded */ TR_UNIT_HAND = 15, /* units 0, 1: o handed off */
+    TR_UNIT_ITEMS = 17, /* unit 0: all partial sums in shared memory */ TR_UNIT_O = 18, /* unit 0: o computed */
+    TR_PUB0 = 25, /* publisher: release of segment k issued and done, k < 7 */
     TR_O_WAIT0 = 19, TR_O_READY0, TR_O_READY_LAST, TR_END, TR_LAST_REDUCE_START, TR_LAST_REDUCE_END,
     TR_TILE_TMA = 32, TR_TILE_MMA = 64, TR_TILE_EPI = 96, TR_TILE_TMA_RET = 128, TR_TILE_ACT = 160 /* per tile i < 32 */
 };
@@ -82,10 +97,19 @@ enum TraceSlot {
 //   (words 2 and 3 are unused)
 //   C_ABORT       set by any wait that gives up
 //   off_oready+kb state units done for o K-block kb (B per step)
-//   off_rb+key    segments published for row block key (q, k, v, o row blocks)
+//   off_rb+key    segments published for row group key (q, k, v, o row groups)
 constexpr int C_XQ = 0, C_GATE = 1, C_ABORT = 4, C_FIXED = 16;
 
+// Status words in mapped host memory: [0] status, [1] wait site, [2] set when a drain of
+// copies in flight gave up (the handle can no longer be trusted).
+constexpr int ST_CODE = 0, ST_WHERE = 1, ST_DRAIN = 2;
+
+constexpr int kOHand = 8;  // o-block hand-off barriers (state unit -> o publisher), reused mod 8
+
 struct __align__(16) VecSmem {
+    uint64_t ohand[kOHand];        // unit k's o planes are stored (arrival of vector warp 0)
+    int opub;                      // units whose o block the o publisher has released
+    int pad_[3];
     float q[256], k[256];          // per head of the unit: q, k^  (heads_per_unit * dk)
     float a[2][256];               // alpha of the current and the next unit (by unit parity)
     float v[128], u[128], o[128];  // per virtual column of the unit
@@ -95,15 +119,17 @@ struct __align__(16) VecSmem {
 };
 
 struct FusedParams {
-    CUtensorMap tm_w[4];  // W_q, W_k, W_v, W_o: uint8 [rows, K], box 128 x 128, 128B swizzle
-    CUtensorMap tm_xq;    // x planes: [2*BP, H], box [2*BP, 128]
+    CUtensorMap tm_w[4];  // W_q, W_k, W_v (box nx rows), W_o (box no rows): uint8 [rows, K], 128B swizzle
+    CUtensorMap tm_xq;    // x planes + scale rows (one box)
+    CUtensorMap tm_xrep;  // one 16-row group of x planes, copied into the empty quarters
     CUtensorMap tm_oq;    // o planes (+ scale rows when they fit in one 256-row box)
-    CUtensorMap tm_osc;   // o scale rows alone, used when 4*BP + scale rows > 256
+    CUtensorMap tm_osc;   // o scale rows alone, used when the o tile is taller than 256 rows
+    CUtensorMap tm_orep;  // one 16-row group of o planes, copied into the empty quarters
     const float *wscale[4];
     const uint16_t *x, *wa_down, *wa_up, *wb;
     float *state;
     void *out;
-    uint8_t *xq, *oq;  // planes + scale rows
+    uint8_t *xq, *oq;  // x and o planes + scale rows
     float *part;
     float *q, *k, *v, *bpre, *t;
     uint32_t *ctr;
@@ -111,14 +137,18 @@ struct FusedParams {
     const TileEntry *tiles;
     const uint32_t *cta_off;
     int *status;
-    const uint2 *rbinfo;  // per row-block key: (first partial slot, segments)
+    const uint2 *rbinfo;  // per row-group key: (first partial slot, segments)
     int B, H, nh, dk, dv, r;
-    int nKBx, nKBo, nRBq, nRBv, nRBo;
+    int nKBx, nKBo, nRGq, nRGv, nRGo;
     int off_oready, off_rb;
     uint32_t epoch, t_xq, t_gate, t_o;
     uint64_t timeout_ns;
-    int out_bf16, stages, stage_bytes, nacc, skip_gate_release;
+    int out_bf16, stages, a_bytes, w_bytes, nacc, cols, skip_gate_release, early_tiles;
 };
+
+// Floats per partial-sum slot: [pair][BP][N <= 256]; pair 1 only for the o planes 2 and 3.
+template <int BP>
+__host__ __device__ constexpr size_t slot_floats() { return (size_t)2 * BP * 256; }
 
 struct Ctl {
     const FusedParams &P;
@@ -146,8 +176,9 @@ __device__ void raise_abort(const Ctl &c, int where)
     *c.sh_abort = 1;
     atomicExch(c.P.ctr + C_ABORT, 1u);
     volatile int *st = c.P.status;  // mapped host memory: plain stores, no atomics
-    st[0] = KDA_ERR_DEVICE_TIMEOUT;
-    st[1] = where;
+    st[ST_WHERE] = where;           // the site first, so a host that sees the code sees its site
+    __threadfence_system();
+    st[ST_CODE] = KDA_ERR_DEVICE_TIMEOUT;
     __threadfence_system();
 }
 
@@ -169,12 +200,19 @@ __device__ bool wait_bar(uint64_t *b, uint32_t parity, const Ctl &c, int where)
     }
 }
 
-// Bounded wait for the phase a barrier is known to reach (used on the exit path only).
-__device__ void drain_bar(uint64_t *b, uint32_t parity, uint64_t limit_ns)
+// Bounded wait for the phase a barrier is known to reach (exit path only).  If it gives up,
+// copies or MMAs of this CTA may still be in flight: record that the handle is unusable.
+__device__ void drain_bar(const FusedParams &P, uint64_t *b, uint32_t parity)
 {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(b, parity))
-        if (globaltimer_ns() - t0 > limit_ns) return;
+    while (!mbar_try_wait(b, parity)) {
+        if (globaltimer_ns() - t0 > P.timeout_ns) {
+            volatile int *st = P.status;
+            st[ST_DRAIN] = 1;
+            __threadfence_system();
+            return;
+        }
+    }
 }
 
 __device__ bool wait_count(const uint32_t *p, uint32_t target, const Ctl &c, int where)
@@ -194,40 +232,24 @@ __device__ bool wait_count(const uint32_t *p, uint32_t target, const Ctl &c, int
     }
 }
 
-__device__ __forceinline__ int rb_key(const FusedParams &P, int mat, int rb)
+__device__ __forceinline__ int rg_key(const FusedParams &P, int mat, int rg)
 {
-    return mat < 2 ? mat * P.nRBq + rb : (mat == 2 ? 2 * P.nRBq + rb : 2 * P.nRBq + P.nRBv + rb);
+    return mat < 2 ? mat * P.nRGq + rg : (mat == 2 ? 2 * P.nRGq + rg : 2 * P.nRGq + P.nRGv + rg);
 }
 
-// Sum of the published partials of row `r` (0..127), sequence b, of row block `key`, in slot order.
+// Two sums over the segments of a row group, element `off` of each slot, in slot order, with
+// all loads of 8 slots per item issued together; items with has[j] false are skipped.
 template <int BP>
-__device__ __forceinline__ float sum_partials(const FusedParams &P, int key, int b, int r)
+__device__ __forceinline__ void sum_segs2(const FusedParams &P, const int (&key)[2], const int (&off)[2],
+                                          const bool (&has)[2], float (&out)[2])
 {
-    const uint2 info = __ldg(P.rbinfo + key);
-    const float *base = P.part + ((size_t)info.x * BP + b) * 128 + r;
-    float s = 0.f;
-    for (uint32_t g0 = 0; g0 < info.y; g0 += 8) {
-        float v[8];
-#pragma unroll
-        for (int g = 0; g < 8; ++g) v[g] = g0 + g < info.y ? __ldcg(base + (size_t)(g0 + g) * BP * 128) : 0.f;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) s += v[g];
-    }
-    return s;
-}
-
-// Two sums of the kind above with all their loads issued together (8 slots per item at a
-// time); items with has[j] false are skipped.  Same slot order, so the same bits.
-template <int BP>
-__device__ __forceinline__ void sum_partials2(const FusedParams &P, const int (&key)[2], const int (&r)[2],
-                                              const bool (&has)[2], int b, float (&out)[2])
-{
+    constexpr size_t SLOT = slot_floats<BP>();
     uint2 info[2];
     const float *base[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         info[j] = has[j] ? __ldg(P.rbinfo + key[j]) : make_uint2(0u, 0u);
-        base[j] = P.part + ((size_t)info[j].x * BP + b) * 128 + r[j];
+        base[j] = P.part + (size_t)info[j].x * SLOT + off[j];
         out[j] = 0.f;
     }
     const uint32_t nmax = info[0].y > info[1].y ? info[0].y : info[1].y;
@@ -236,8 +258,7 @@ __device__ __forceinline__ void sum_partials2(const FusedParams &P, const int (&
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
-            for (int g = 0; g < 8; ++g)
-                v[j][g] = g0 + g < info[j].y ? __ldcg(base[j] + (size_t)(g0 + g) * BP * 128) : 0.f;
+            for (int g = 0; g < 8; ++g) v[j][g] = g0 + g < info[j].y ? __ldcg(base[j] + (size_t)(g0 + g) * SLOT) : 0.f;
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -262,14 +283,22 @@ __device__ __forceinline__ float pow2_scale(float amax)
     return ldexpf(1.f, m == 0.5f ? e - 1 : e);
 }
 
-// Plane buffers hold, per K block (128 bytes of every row), NP planes of BP rows and then
-// the BP fp32 scales of the block in ceil(BP/32) extra rows ("scale rows"), so one TMA
-// copy brings a tile's activation planes and their scales.
-__host__ __device__ constexpr int scale_rows(int BP) { return (BP + 31) / 32; }
-__device__ __forceinline__ float *scale_slot(uint8_t *rowbase0, size_t pitch, int NP, int BP, int b)
+// Row of plane p of sequence b in an x tile (2 planes; group b / 8) and in an o tile (4
+// planes; group 2 (b / 8) + p / 2).
+__device__ __forceinline__ int x_row(int p, int b) { return act_rowbase(b / 8) + 8 * p + (b % 8); }
+__device__ __forceinline__ int o_row(int p, int b) { return act_rowbase(2 * (b / 8) + p / 2) + 8 * (p % 2) + (b % 8); }
+
+// Rows of the first TMA box of an activation tile with `groups` groups: its groups and
+// scale rows, at most 256 rows (the scale rows past 256 come in a second box).
+__host__ __device__ constexpr int act_main_rows(int groups, int sr)
 {
-    return reinterpret_cast<float *>(rowbase0 + (size_t)(NP * BP + b / 32) * pitch + (b % 32) * 4);
+    return groups <= 4 ? (act_rowbase(groups - 1) + 16 > 16 + sr ? act_rowbase(groups - 1) + 16 : 16 + sr)
+                       : (act_rows(groups, sr) > 256 ? 256 : act_rows(groups, sr));
 }
+
+// Byte offset of (row r, byte c) in a 128-byte-swizzled tile: 16-byte chunk c / 16 of row r
+// sits at chunk (c / 16) ^ (r % 8).
+__device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((((c >> 4) ^ (r & 7))) << 4) + (c & 15); }
 
 // Splits four values (already divided by their scale) into NP E4M3 planes, 4 codes per word.
 template <int NP>
@@ -325,6 +354,7 @@ __device__ __forceinline__ void prefetch_l2_slice(const void *p, size_t bytes)
 template <int BP>
 __device__ void quantize_x(const FusedParams &P, int gw, int ngw, int lane)
 {
+    constexpr ActGeo G = act_geo(BP);
     const int items = P.B * P.nKBx;
     for (int it = gw; it < items; it += ngw) {
         const int b = it / P.nKBx, kb = it % P.nKBx;
@@ -337,8 +367,9 @@ __device__ void quantize_x(const FusedParams &P, int gw, int ngw, int lane)
         split_planes<2>(v0 * inv, v1 * inv, v2 * inv, v3 * inv, w);
 #pragma unroll
         for (int p = 0; p < 2; ++p)
-            *reinterpret_cast<uint32_t *>(P.xq + (size_t)(p * BP + b) * P.H + kb * 128 + lane * 4) = w[p];
-        if (lane == 0) *scale_slot(P.xq + kb * 128, P.H, 2, BP, b) = s;
+            *reinterpret_cast<uint32_t *>(P.xq + (size_t)x_row(p, b) * P.H + kb * 128 + lane * 4) = w[p];
+        if (lane == 0)
+            *reinterpret_cast<float *>(P.xq + (size_t)(G.rsx + b / 32) * P.H + kb * 128 + (b % 32) * 4) = s;
         fence_proxy_async_global();
         __syncwarp();
         if (lane == 0) red_release_add(P.ctr + C_XQ, 1u);
@@ -444,12 +475,65 @@ __device__ void unit_gates(const FusedParams &P, VecSmem *vs, int u, int slot, i
     }
 }
 
+// Gates of this CTA's first two units (u1 < 0: none) into slots 0 and 1, by all 256 vector
+// threads with every load issued in one batch: t of the two sequences into shared memory,
+// beta, and one W_a_up row per thread and unit.  t and W_b x must be final.
+template <int DK>
+__device__ void first_gates(const FusedParams &P, VecSmem *vs, int u0, int u1, int vt)
+{
+    const int hpu = 128 / P.dv, rows = hpu * DK, r4 = P.r / 4;
+    const int us[2] = {u0, u1};
+    float *ts = &vs->red_w[0][0];  // [2][r] (r <= 256)
+    if (vt < 2 * r4) {
+        const int j = vt / r4, c4 = vt % r4;
+        if (us[j] >= 0)
+            *reinterpret_cast<float4 *>(ts + j * P.r + 4 * c4) =
+                __ldcg(reinterpret_cast<const float4 *>(P.t + (size_t)(us[j] % P.B) * P.r) + c4);
+    } else if (vt >= 128 && vt < 128 + 2 * hpu) {
+        const int j = (vt - 128) / hpu, hh = (vt - 128) % hpu;
+        if (us[j] >= 0) {
+            const int b = us[j] % P.B, h = (us[j] / P.B) * hpu + hh;
+            vs->beta[j][hh] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h)));
+        }
+    }
+    for (int idx0 = 0; idx0 < 2 * rows; idx0 += 256) {
+        const int idx = idx0 + vt, j = idx / rows, i = idx % rows;
+        const bool has = idx < 2 * rows && us[j < 2 ? j : 0] >= 0;
+        const uint16_t *wr = P.wa_up + ((size_t)((has ? us[j] : 0) / P.B) * hpu * DK + i) * P.r;
+        float z = 0.f;
+        for (int j0 = 0; j0 < P.r; j0 += 64) {
+            uint4 w4[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                w4[q] = has && j0 + q * 8 < P.r ? __ldg(reinterpret_cast<const uint4 *>(wr + j0 + q * 8))
+                                                : make_uint4(0, 0, 0, 0);
+            if (j0 == 0) named_bar(2, 256);  // t is in shared memory
+            if (has) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (j0 + q * 8 >= P.r) break;
+                    const uint32_t wv[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
+                    const float *tv = ts + j * P.r + j0 + q * 8;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        z = fmaf(bf16_bits_to_float(wv[e] & 0xFFFFu), tv[2 * e], z);
+                        z = fmaf(bf16_bits_to_float(wv[e] >> 16), tv[2 * e + 1], z);
+                    }
+                }
+            }
+        }
+        if (has) vs->a[j][i] = 1.f / (1.f + expf(z));
+    }
+    named_bar(2, 256);
+}
+
 // One state unit: sequence b, o K-block kb (heads kb*128/dv ..), all dk rows.  Its gates are
-// in slot nu & 1; while warp 0 waits for the unit's q/k/v, warps 1-7 compute the gates of
-// this CTA's next unit (next_u >= 0) into the other slot.
+// in slot nu & 1; while a few threads wait for the unit's q/k/v, the others compute the gates
+// of this CTA's next unit (next_u >= 0) into the other slot.
 template <int BP, int DK>
 __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int u, int next_u, int vt, int nu)
 {
+    constexpr ActGeo G = act_geo(BP);
     const int b = u % P.B, kb = u / P.B, slot = nu & 1;
     constexpr int RPW = DK / 8;  // rows per warp
     const int vw = vt >> 5, lane = vt & 31;
@@ -464,15 +548,17 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 
     if (vt == 0) vs->fail = 0;
     named_bar(2, 256);
-    // then the heads' q, k, v: wait for every segment of their row blocks (one thread per
+    // then the heads' q, k, v: wait for every segment of their row groups (one thread per
     // counter, so the round trips overlap), add the partials
     {
-        const int rlo = h0 * DK / 128, nq = ((h0 + hpu) * DK - 1) / 128 - rlo + 1;
-        if (vt < 2 * nq + 1) {
-            const int key = vt < nq ? rlo + vt : (vt < 2 * nq ? P.nRBq + rlo + (vt - nq) : 2 * P.nRBq + kb);
+        const int glo = h0 * DK / G.nx, nq = ((h0 + hpu) * DK - 1) / G.nx - glo + 1;
+        const int vlo = kb * 128 / G.nx, nv = (kb * 128 + 127) / G.nx - vlo + 1;
+        if (vt < 2 * nq + nv) {
+            const int key = vt < nq ? glo + vt
+                                    : (vt < 2 * nq ? P.nRGq + glo + (vt - nq) : 2 * P.nRGq + vlo + (vt - 2 * nq));
             if (!wait_rb(P, key, c, 11)) vs->fail = 1;
         }
-        if (next_u >= 0) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
+        if (next_u >= 0 && nu >= 1) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
     }
     named_bar(2, 256);
     if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
@@ -481,25 +567,27 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         // items: q and k rows of the unit's heads, then its 128 v columns; a thread's items
         // are loaded together (one memory round trip), then summed in slot order
         const int nqk = hpu * DK, nitems = 2 * nqk + 128;
-        for (int it0 = 0; it0 < nitems; it0 += 512) {  // 384 items (dk = 128) or 640 (dk = 128, dv = 64)
-            int key[2], r[2];
+        for (int it0 = 0; it0 < nitems; it0 += 512) {
+            int key[2], off[2];
             bool has[2];
-    #pragma unroll
+#pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int it = it0 + vt + 256 * j;
                 has[j] = it < nitems;
                 if (it < 2 * nqk) {
                     const int row = h0 * DK + it % nqk;
-                    key[j] = (it / nqk) * P.nRBq + row / 128;
-                    r[j] = row % 128;
+                    key[j] = (it / nqk) * P.nRGq + row / G.nx;
+                    off[j] = b * G.nx + row % G.nx;
                 } else {
-                    key[j] = 2 * P.nRBq + kb;
-                    r[j] = it - 2 * nqk;
+                    const int col = kb * 128 + (it - 2 * nqk);
+                    key[j] = 2 * P.nRGq + col / G.nx;
+                    off[j] = b * G.nx + col % G.nx;
                 }
             }
             float val[2];
-            sum_partials2<BP>(P, key, r, has, b, val);
-    #pragma unroll
+            sum_segs2<BP>(P, key, off, has, val);
+            if (vt == 0 && nu < 2 && it0 == 0) KDA_TR(P, TR_UNIT_SUMS + nu);
+#pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int it = it0 + vt + 256 * j;
                 if (!has[j]) continue;
@@ -516,6 +604,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         }
     }
     named_bar(2, 256);
+    if (vt == 0 && nu == 0) KDA_TR(P, TR_UNIT_ITEMS);
     // ||k|| and k.q per head (one warp per head)
     if (vw < hpu) {
         float ss = 0.f, kq = 0.f;
@@ -564,6 +653,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         vs->o[vt] = fmaf(uu, vs->kq[hx], p);
     }
     named_bar(2, 256);
+    if (vt == 0 && nu == 0) KDA_TR(P, TR_UNIT_O);
     // o -> four E4M3 planes with one power-of-two scale for the K-block; release it
     if (vw == 0) {
         const float4 o4 = *reinterpret_cast<const float4 *>(&vs->o[vc]);
@@ -573,13 +663,21 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         split_planes<4>(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv, wq);
 #pragma unroll
         for (int p = 0; p < 4; ++p)
-            *reinterpret_cast<uint32_t *>(P.oq + (size_t)(p * BP + b) * Dv + (size_t)kb * 128 + vc) = wq[p];
-        if (lane == 0) *scale_slot(P.oq + (size_t)kb * 128, Dv, 4, BP, b) = sc;
+            *reinterpret_cast<uint32_t *>(P.oq + (size_t)o_row(p, b) * Dv + (size_t)kb * 128 + vc) = wq[p];
+        if (lane == 0)
+            *reinterpret_cast<float *>(P.oq + (size_t)(G.rso + b / 32) * Dv + (size_t)kb * 128 + (b % 32) * 4) = sc;
         fence_proxy_async_global();
         __syncwarp();
-        if (lane == 0) red_release_add(P.ctr + P.off_oready + kb, 1u);
+        if (lane == 0) {
+            // hand the release to the o publisher (its fence then never holds up the unit); at
+            // most kOHand units may wait for it
+            const uint64_t t0 = globaltimer_ns();
+            while (nu - *(volatile int *)&vs->opub >= kOHand && globaltimer_ns() - t0 < P.timeout_ns) __nanosleep(64);
+            mbar_arrive(&vs->ohand[nu % kOHand]);
+            if (nu < 2) KDA_TR(P, TR_UNIT_HAND + nu);
+        }
     }
-    // S' = S~ + k^ u^T, written back in place (after the release: nothing reads it this step)
+    // S' = S~ + k^ u^T, written back in place (after the hand-off: nothing reads it this step)
     const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
 #pragma unroll
     for (int r = 0; r < RPW; ++r) {
@@ -593,28 +691,39 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
     return true;
 }
 
+// Warp 1, lane 0: releases the o blocks of this CTA's state units, in unit order, once vector
+// warp 0 has stored their planes.
+__device__ void o_publisher(const FusedParams &P, VecSmem *vs, const Ctl &c)
+{
+    const int units = P.B * P.nKBo;
+    for (int k = 0, u = blockIdx.x; u < units; ++k, u += gridDim.x) {
+        if (!wait_bar(&vs->ohand[k % kOHand], (uint32_t)(k / kOHand) & 1u, c, 14)) return;
+        if (!*c.sh_abort) red_release_add(P.ctr + P.off_oready + u / P.B, 1u);
+        *(volatile int *)&vs->opub = k + 1;
+    }
+}
+
+// State of unit u (sequence u % B, the heads of o K-block u / B) -> L2, in 32 KB bulk prefetches.
+__device__ void prefetch_unit_state(const FusedParams &P, int u)
+{
+    const int b = u % P.B, kb = u / P.B, hpu = 128 / P.dv;
+    const size_t bytes = (size_t)hpu * P.dk * P.dv * 4;
+    const char *p = reinterpret_cast<const char *>(P.state + (((size_t)b * P.nh + (size_t)kb * hpu) * P.dk) * P.dv);
+    const uint64_t pol = policy_evict_last();
+    for (size_t o = 0; o < bytes; o += 32768)
+        bulk_prefetch_l2_hint(p + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
+}
+
 template <int BP, int DK>
 __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
 {
+    constexpr ActGeo G = act_geo(BP);
     const int vt = threadIdx.x - 256, vw = vt >> 5, lane = vt & 31;
-    const int gw = blockIdx.x * 8 + vw, ngw = gridDim.x * 8;
-    quantize_x<BP>(P, gw, ngw, lane);
+    quantize_x<BP>(P, blockIdx.x * 8 + vw, gridDim.x * 8, lane);
     if (vt == 0) KDA_TR(P, TR_XQ_DONE);
+    if (vt == 0 && (int)blockIdx.x < P.B * P.nKBo) prefetch_unit_state(P, blockIdx.x);
     gate_rows<BP>(P, vs, vt);
     if (vt == 0) KDA_TR(P, TR_GATES_DONE);
-    if (vt == 0) {
-        // warm L2 with this CTA's share of the recurrent state: units read it from L2 later
-        const size_t sbytes = (size_t)P.B * P.nh * P.dk * P.dv * 4;
-        const size_t gran = (sbytes / 16 + gridDim.x - 1) / gridDim.x * 16;
-        const size_t lo = (size_t)blockIdx.x * gran;
-        if (lo < sbytes) {
-            const size_t nb = (sbytes - lo < gran ? sbytes - lo : gran) & ~(size_t)15;
-            const uint64_t pol = policy_evict_last();
-            for (size_t o = 0; o < nb; o += 32768)
-                bulk_prefetch_l2_hint(reinterpret_cast<const char *>(P.state) + lo + o,
-                                      (uint32_t)(nb - o < 32768 ? nb - o : 32768), pol);
-        }
-    }
     // State units (sequence u % B, o K-block u / B) in head order, CTA c taking c, c + grid,
     // ...: the same units every step, so the next unit's gates are computed while the
     // current one waits for its q/k/v.
@@ -623,8 +732,8 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
         if (vt == 0) vs->ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);  // t and W_b x final
         named_bar(2, 256);
         if (!vs->ok) return;
-        unit_gates<DK>(P, vs, blockIdx.x, 0, vt, 0, 256);
-        named_bar(2, 256);
+        const int u1 = (int)(blockIdx.x + gridDim.x);
+        first_gates<DK>(P, vs, blockIdx.x, u1 < units ? u1 : -1, vt);
     }
     for (int nu = 0, u = blockIdx.x; u < units; ++nu, u += gridDim.x) {
         if (vt == 0) vs->unit = should_stop(c) ? 1 : 0;
@@ -632,18 +741,23 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
         if (vs->unit) return;
         if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu);
         const int next = u + (int)gridDim.x < units ? u + (int)gridDim.x : -1;
+        if (vt == 0 && next >= 0) prefetch_unit_state(P, next);  // its state streams in meanwhile
         if (!state_unit<BP, DK>(P, vs, c, u, next, vt, nu)) return;
         if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
     }
-    // out = sum of the W_o partials: items of (row block, 32-row quarter)
-    for (int item = blockIdx.x; item < 4 * P.nRBo; item += gridDim.x) {
-        const int rb = item >> 2, key = 2 * P.nRBq + P.nRBv + rb;
+    // out = sum of the W_o partials (both plane pairs): items of 32 output rows
+    for (int item = blockIdx.x; item < P.H / 32; item += gridDim.x) {
+        const int grow0 = item * 32, rg = grow0 / G.no, key = 2 * P.nRGq + P.nRGv + rg;
         if (vt == 0) vs->ok = wait_rb(P, key, c, 12);
         named_bar(2, 256);
         if (!vs->ok) return;
-        const int r = (item & 3) * 32 + lane, grow = rb * 128 + r;
+        const int grow = grow0 + lane, n = grow % G.no;
         for (int b = vw; b < P.B; b += 8) {
-            const float v = sum_partials<BP>(P, key, b, r);
+            const int kk[2] = {key, key}, off[2] = {b * G.no + n, (BP + b) * G.no + n};
+            const bool has[2] = {true, true};
+            float val[2];
+            sum_segs2<BP>(P, kk, off, has, val);
+            const float v = val[0] + val[1];
             if (P.out_bf16) static_cast<__nv_bfloat16 *>(P.out)[(size_t)b * P.H + grow] = __float2bfloat16_rn(v);
             else static_cast<float *>(P.out)[(size_t)b * P.H + grow] = v;
         }
@@ -653,33 +767,71 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
 
 // ---------------------------------------------------------------- projection pipeline
 
-// Shared-memory ring.  Stage s holds the weight tile (16 KB), the activation planes of the
-// same tile (up to 4 planes x BP rows x 128 bytes) and their BP scales; one producer issues
-// both copies back to back, so they sit next to each other in the TMA queue.
+// Shared-memory ring.  Stage s: an activation region (1024-aligned), then a weight region.
+// The MMA reads 128 activation rows from a region's start; rows past the ones loaded are junk
+// (the stage's weights), which only fill accumulator lanes nobody reads.
 struct Ring {
-    uint8_t *base;
-    int S, sbytes, NACC;
-    uint64_t *full, *empty, *accfull, *accempty;
-    __device__ uint8_t *w(int s) const { return base + (size_t)s * sbytes; }
-    __device__ uint8_t *a(int s) const { return base + (size_t)s * sbytes + kTileBytes; }
-    // scale of sequence b in the staged activation tile: row NP*BP + b/32 of a 128B-swizzled
-    // tile, 16-byte chunk ((b%32)/4) XOR (row % 8)
-    __device__ float scale(int s, int NP, int BP, int b) const
-    {
-        const int row = NP * BP + b / 32, chunk = ((b % 32) >> 2) ^ (row & 7);
-        return *reinterpret_cast<const float *>(a(s) + row * 128 + chunk * 16 + (b & 3) * 4);
-    }
+    uint8_t *a0;
+    int S, a_bytes, w_bytes, nacc, cols;
+    uint64_t *full, *mmad, *empty, *accempty, *segdone;
+    __device__ uint8_t *a(int s) const { return a0 + (size_t)s * (a_bytes + w_bytes); }
+    __device__ uint8_t *w(int s) const { return a0 + (size_t)s * (a_bytes + w_bytes) + a_bytes; }
 };
+
+// fp32 scale of sequence b in an activation tile whose scale rows start at row R.
+__device__ __forceinline__ float staged_scale(const uint8_t *a, int R, int b)
+{
+    return *reinterpret_cast<const float *>(a + swz(R + b / 32, (b % 32) * 4));
+}
+
+// One activation tile into stage s: the first box (groups and scale rows, up to 256 rows),
+// the scale rows past 256, and a 16-row copy of group v % groups into each empty slot v.
+template <int GR, int SR>
+__device__ __forceinline__ uint32_t act_copy(uint8_t *dst, const CUtensorMap *main, const CUtensorMap *sc,
+                                             const CUtensorMap *rep, int kb, uint64_t *bar, uint64_t pol)
+{
+    constexpr int RO = act_rows(GR, SR), RMAIN = act_main_rows(GR, SR), RSC = RO > 256 ? RO - 256 : 0;
+    constexpr int NREP = act_slots(GR) - GR;
+    const uint32_t bytes = (uint32_t)(RMAIN + RSC + 16 * NREP) * 128u;
+    mbar_expect_tx(bar, bytes);
+    tma_load_2d(dst, main, kb * 128, 0, bar, pol);
+    if (RSC > 0) tma_load_2d(dst + 256 * 128, sc, kb * 128, 256, bar, pol);
+#pragma unroll
+    for (int v = GR; v < GR + NREP; ++v)
+        tma_load_2d(dst + act_rowbase(v) * 128, rep, kb * 128, act_rowbase(v % GR), bar, pol);
+    return bytes;
+}
 
 // Warp 0, lane 0.  Weight copies run up to S tiles ahead; the activation copy of tile i is
 // issued right after its weight copy once its input is final (x split into planes, or an
 // o K-block whose state units are done).  An activation that is not ready yet is deferred
 // and polled only when no weight copy can be issued, so weights keep streaming.
 template <int BP>
-__device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *my, int n, const Ctl &c)
+__device__ __forceinline__ void weight_copy(const FusedParams &P, const Ring &R, const TileEntry &e, int i, uint64_t pol)
 {
+    constexpr ActGeo G = act_geo(BP);
+    const int N = e.mat < 3 ? G.nx : G.no;
+    if (i < 32) KDA_TR(P, TR_TILE_TMA + i);
+    mbar_expect_tx(&R.full[i % R.S], N * 128);
+    tma_load_2d(R.w(i % R.S), &P.tm_w[e.mat], e.kb * 128, e.rg * N, &R.full[i % R.S], pol);
+}
+
+// The weight copies of the first stages (all free at launch); returns how many were issued.
+template <int BP>
+__device__ int preissue_weights(const FusedParams &P, const Ring &R, const TileEntry *my, int n)
+{
+    const uint64_t pol_w = policy_evict_first();
+    const int k = n < R.S ? n : R.S;
+    for (int i = 0; i < k; ++i) weight_copy<BP>(P, R, my[i], i, pol_w);
+    return k;
+}
+
+template <int BP>
+__device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *my, int n, const Ctl &c, int pre)
+{
+    constexpr ActGeo G = act_geo(BP);
     const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
-    int nw = 0, na = 0;  // weight copies issued, activation copies issued (na <= nw)
+    int nw = pre, na = 0;  // weight copies issued, activation copies issued (na <= nw)
     bool x_ok = false;
     uint32_t o_ok[16] = {};  // bit kb: o K-block kb known final (kb < 512)
     uint64_t t_stall = 0, t_poll = 0, t_abort = globaltimer_ns() + 20000;
@@ -699,13 +851,13 @@ __device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *m
         fence_proxy_async_global();  // planes written by other SMs, read by the async proxy
         return true;
     };
-    // Hold the weight stream back after the first kEarlyTiles copies until x is split into
+    // Hold the weight stream back after the first early_tiles copies until x is split into
     // planes (or kEarlyHoldNs passed): the x loads of the splitting CTAs then do not queue
     // behind a full ring of weight copies from every SM, and the MMA starts sooner.
     const uint64_t hold_until = globaltimer_ns() + kEarlyHoldNs;
     while (na < n) {
         bool progress = false;
-        if (!x_ok && nw >= kEarlyTiles && nw < n && my[nw].mat < 3 && globaltimer_ns() < hold_until) {
+        if (!x_ok && nw >= P.early_tiles && nw < n && my[nw].mat < 3 && globaltimer_ns() < hold_until) {
             if (!poll_ready(my[nw])) {
                 __nanosleep(128);
                 continue;
@@ -713,22 +865,16 @@ __device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *m
         }
         while (na < nw && known_ready(my[na])) {
             const TileEntry e = my[na];
-            const int s = na % R.S;
-            const int np = e.mat < 3 ? 2 : 4;
+            uint64_t *bar = &R.full[na % R.S];
+            uint8_t *dst = R.a(na % R.S);
             if (na < 32) KDA_TR(P, TR_TILE_ACT + na);
-            mbar_expect_tx(&R.full[s], (np * BP + scale_rows(BP)) * 128);
-            tma_load_2d(R.a(s), e.mat < 3 ? &P.tm_xq : &P.tm_oq, e.kb * 128, 0, &R.full[s], pol_a);
-            if (e.mat == 3 && 4 * BP + scale_rows(BP) > 256)
-                tma_load_2d(R.a(s) + 4 * BP * 128, &P.tm_osc, e.kb * 128, 4 * BP, &R.full[s], pol_a);
+            if (e.mat < 3) act_copy<G.gx, G.sr>(dst, &P.tm_xq, &P.tm_xq, &P.tm_xrep, e.kb, bar, pol_a);
+            else act_copy<G.go, G.sr>(dst, &P.tm_oq, &P.tm_osc, &P.tm_orep, e.kb, bar, pol_a);
             ++na;
             progress = true;
         }
         if (nw < n && nw - na < R.S && mbar_test_wait(&R.empty[nw % R.S], ((uint32_t)(nw / R.S) & 1u) ^ 1u)) {
-            const TileEntry e = my[nw];
-            if (nw < 32) KDA_TR(P, TR_TILE_TMA + nw);
-            mbar_expect_tx(&R.full[nw % R.S], kTileBytes);
-            tma_load_2d(R.w(nw % R.S), &P.tm_w[e.mat], e.kb * 128, e.rb * 128, &R.full[nw % R.S], pol_w);
-            if (nw < 32) KDA_TR(P, TR_TILE_TMA_RET + nw);
+            weight_copy<BP>(P, R, my[nw], nw, pol_w);
             ++nw;
             t_stall = 0;
             continue;
@@ -753,60 +899,125 @@ __device__ void producer(const FusedParams &P, const Ring &R, const TileEntry *m
     // Every issued copy must land before the CTA may exit.  Stages whose activation copy was
     // never issued get the missing arrival, so their phase completes when the weight lands.
     for (int i = na; i < nw; ++i) mbar_arrive(&R.full[i % R.S]);
-    for (int i = nw > R.S ? nw - R.S : 0; i < nw; ++i)
-        drain_bar(&R.full[i % R.S], (uint32_t)(i / R.S) & 1u, P.timeout_ns);
+    for (int i = nw > R.S ? nw - R.S : 0; i < nw; ++i) drain_bar(P, &R.full[i % R.S], (uint32_t)(i / R.S) & 1u);
 }
 
 template <int BP>
 __device__ void mma_issuer(const FusedParams &P, const Ring &R, const TileEntry *my, int n, uint32_t tmem,
                            const Ctl &c)
 {
+    constexpr ActGeo G = act_geo(BP);
     int issued = 0;
     for (int i = 0; i < n; ++i) {
         const TileEntry e = my[i];
-        const int s = i % R.S, buf = i % R.NACC;
-        const uint32_t ph = (uint32_t)(i / R.S) & 1u, bph = (uint32_t)(i / R.NACC) & 1u;
-        if (!wait_bar(&R.full[s], ph, c, 5)) break;
-        if (!wait_bar(&R.accempty[buf], bph ^ 1u, c, 7)) break;
+        const int s = i % R.S, buf = i % R.nacc;
+        if (!wait_bar(&R.full[s], (uint32_t)(i / R.S) & 1u, c, 5)) break;
+        if (i >= R.nacc && !wait_bar(&R.accempty[buf], ((uint32_t)(i / R.nacc) & 1u) ^ 1u, c, 7)) break;
         tc_fence_after();
-        const uint32_t idesc = e.mat < 3 ? idesc_e4m3_f32(128, 2 * BP) : idesc_e4m3_f32(128, 4 * BP);
-        const uint32_t aa = smem_u32(R.w(s)), ba = smem_u32(R.a(s));
-        const uint32_t d = tmem + (uint32_t)(buf * 4 * BP);
+        const bool isx = e.mat < 3;
+        const int N = isx ? G.nx : G.no, MH = isx ? G.mhx : G.mho;
+        const uint32_t idesc = idesc_e4m3_f32(128, (uint32_t)N);
+        const uint32_t aa = smem_u32(R.a(s)), wa = smem_u32(R.w(s));
+        const uint32_t d = tmem + (uint32_t)(buf * R.cols);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            mma_f8f6f4(d, sdesc_k128_sw128(aa + ks * 32), sdesc_k128_sw128(ba + ks * 32), idesc, ks > 0 ? 1u : 0u);
-        mma_commit(&R.empty[s]);
-        mma_commit(&R.accfull[buf]);
+            for (int h = 0; h < MH; ++h)
+                mma_f8f6f4(d + (uint32_t)(h * N), sdesc_k128_sw128(aa + h * 16384 + ks * 32),
+                           sdesc_k128_sw128(wa + ks * 32), idesc, ks > 0 ? 1u : 0u);
+        mma_commit(&R.mmad[s]);
         if (issued == 0) KDA_TR(P, TR_FIRST_MMA);
         if (i < 32) KDA_TR(P, TR_TILE_MMA + i);
         ++issued;
     }
     if (issued > 0) {  // the last MMAs must finish before TMEM is freed
         const int i = issued - 1;
-        drain_bar(&R.accfull[i % R.NACC], (uint32_t)(i / R.NACC) & 1u, P.timeout_ns);
+        drain_bar(P, &R.mmad[i % R.S], (uint32_t)(i / R.S) & 1u);
     }
 }
 
-template <int NPL, int BP>
-__device__ __forceinline__ void accumulate_tile(uint32_t taddr, const Ring &R, int s, float ws, float (&acc)[BP])
+// 16x256b TMEM load, 8 repetitions: for repetition r, registers 4r, 4r+1 hold lane
+// (base + t/4) and 4r+2, 4r+3 lane (base + 8 + t/4), columns 8r + 2 (t % 4) + {0, 1}.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32])
 {
-    constexpr int N = NPL * BP;
-    constexpr bool kCache = BP <= 32;  // keep the BP combined scales in registers
-    float as[kCache ? BP : 1];
-    if (kCache) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Slots of warp quarter q: v = q, q + 4, ...  Slot v holds row group g = v % GR (x: sequences
+// 8g..8g+7, planes 0-1; o: sequences 8(g/2).., planes 2(g%2), 2(g%2)+1).  With fewer than
+// four groups, the copies of a group split its N columns: slot v takes part v / GR.
+template <int GR, int N>
+struct EpiGeo {
+    static constexpr int SL = GR < 4 ? 4 : GR;       // slots
+    static constexpr int CS = GR < 4 ? 4 / GR : 1;   // column parts per group
+    static constexpr int NW = N / CS;                // columns per slot
+    static constexpr int GPW = SL / 4;               // slots per warp
+    static constexpr int KPS = NW / 4;               // running sums per slot and thread
+    static_assert(GPW * KPS <= 64, "running sums exceed the register budget");
+    static_assert(NW % 64 == 0, "a slot's columns come in 64-column loads");
+};
+
+// One tile into the running sums of warp quarter q.  Thread t owns sequence (first of the
+// group) + t/4 and KPS columns; both of its planes arrive in the same load and are added
+// before the scale.
+template <int GR, int N, bool O>
+__device__ __forceinline__ void epi_accumulate(uint32_t tq, int q, int t, const uint8_t *as, int RS, float fw0,
+                                               float fw1, float (&acc)[64])
+{
+    using E = EpiGeo<GR, N>;
 #pragma unroll
-        for (int b = 0; b < (kCache ? BP : 1); ++b) as[b] = ws * R.scale(s, NPL, BP, b);
+    for (int gi = 0; gi < E::GPW; ++gi) {
+        const int v = q + 4 * gi, g = v % GR, part = v / GR;
+        if (v < E::SL) {
+            const int h = v / 8;
+            const uint32_t lofs = (uint32_t)(16 * ((v % 8) / 4));
+            const int b = (O ? 8 * (g / 2) : 8 * g) + (t >> 2);
+            const float sa = staged_scale(as, RS, b);
+            const float f0 = fw0 * sa, f1 = fw1 * sa;
+            const int col0 = GR < 4 ? part * E::NW : 0;
+#pragma unroll
+            for (int c8 = 0; c8 < E::NW / 64; ++c8) {
+                uint32_t r[32];
+                tmem_ld_16x256b_x8(tq + (lofs << 16) + (uint32_t)(h * N + col0 + c8 * 64), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int rep = 0; rep < 8; ++rep) {
+                    const float f = (col0 + c8 * 64 + rep * 8 < 128) ? f0 : f1;
+                    const int k = gi * E::KPS + (c8 * 8 + rep) * 2;
+                    acc[k] = fmaf(f, __uint_as_float(r[4 * rep]) + __uint_as_float(r[4 * rep + 2]), acc[k]);
+                    acc[k + 1] = fmaf(f, __uint_as_float(r[4 * rep + 1]) + __uint_as_float(r[4 * rep + 3]), acc[k + 1]);
+                }
+            }
+        }
     }
+}
+
+// The running sums of warp quarter q -> partial-sum slot [pair][BP][N].
+template <int BP, int GR, int N, bool O>
+__device__ __forceinline__ void epi_publish(float *slot, int q, int t, int B, const float (&acc)[64])
+{
+    using E = EpiGeo<GR, N>;
 #pragma unroll
-    for (int c0 = 0; c0 < N; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + (uint32_t)c0, v);
-        tmem_wait_ld();
+    for (int gi = 0; gi < E::GPW; ++gi) {
+        const int v = q + 4 * gi, g = v % GR, part = v / GR;
+        if (v < E::SL) {
+            const int b = (O ? 8 * (g / 2) : 8 * g) + (t >> 2), pair = O ? (g & 1) : 0;
+            const int col0 = GR < 4 ? part * E::NW : 0;
+            if (b < B) {
+                float *dst = slot + ((size_t)pair * BP + b) * N + col0 + 2 * (t & 3);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int b = (c0 + j) % BP;
-            const float f = kCache ? as[kCache ? b : 0] : ws * R.scale(s, NPL, BP, b);
-            acc[b] = fmaf(f, v[j], acc[b]);
+                for (int cc = 0; cc < E::NW / 8; ++cc) {
+                    const int k = gi * E::KPS + 2 * cc;
+                    __stcg(reinterpret_cast<float2 *>(dst + 8 * cc), make_float2(acc[k], acc[k + 1]));
+                }
+            }
         }
     }
 }
@@ -820,58 +1031,81 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t *b, uint32_t parity, cons
 }
 
 // Warps 4-7: per tile, read the fp32 accumulator from TMEM, scale it and add it to the
-// running segment sum in registers; at a segment end publish the partial and release it.
-// Nothing here waits on global memory, so the MMA (up to NACC buffers ahead) never idles
-// behind a publication.  After an abort the loop keeps running with the work skipped, so
-// that all 128 threads pass the same named barriers.
+// running segment sums in registers; at a segment end store the partials and hand the
+// segment to the publisher.  Nothing here waits on global memory, so the MMA (up to nacc
+// buffers ahead) never idles behind a publication.  After an abort the loop keeps running
+// with the work skipped, so that the publisher still sees every hand-off.
 template <int BP>
 __device__ void epilogue_role(const FusedParams &P, const Ring &R, const TileEntry *my, int n, uint32_t tmem,
                               const Ctl &c)
 {
-    const int et = threadIdx.x - 128;  // 0..127
-    const int quarter = (threadIdx.x >> 5) & 3;
-    const int lane = threadIdx.x & 31;
-    const int row = quarter * 32 + lane;  // TMEM lane = weight row within the tile
-    const uint32_t taddr_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    constexpr ActGeo G = act_geo(BP);
+    const int q = ((int)threadIdx.x >> 5) & 3;  // TMEM lane quarter of this warp
+    const int t = threadIdx.x & 31;
+    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
     bool dead = false;
-    float acc[BP];
+    int nseg = 0;
+    float acc[64];
 #pragma unroll
-    for (int b = 0; b < BP; ++b) acc[b] = 0.f;
-    auto wscale_of = [&](const TileEntry &t) {
-        return __ldg(P.wscale[t.mat] + (size_t)t.rb * (t.mat < 3 ? P.nKBx : P.nKBo) + t.kb);
+    for (int k = 0; k < 64; ++k) acc[k] = 0.f;
+    auto wscales = [&](const TileEntry &e, float &w0, float &w1) {
+        const int N = e.mat < 3 ? G.nx : G.no;
+        const int rows = e.mat < 2 ? P.nh * P.dk : (e.mat == 2 ? P.nh * P.dv : P.H);
+        const int nkb = e.mat < 3 ? P.nKBx : P.nKBo, rb0 = e.rg * N / 128;
+        w0 = __ldg(P.wscale[e.mat] + (size_t)rb0 * nkb + e.kb);
+        w1 = (N == 256 && (rb0 + 1) * 128 < rows) ? __ldg(P.wscale[e.mat] + (size_t)(rb0 + 1) * nkb + e.kb) : 0.f;
     };
-    float ws_next = n > 0 ? wscale_of(my[0]) : 0.f;
+    float w0n = 0.f, w1n = 0.f;
+    if (n > 0) wscales(my[0], w0n, w1n);
     for (int i = 0; i < n; ++i) {
         const TileEntry e = my[i];
-        const int s = i % R.S, buf = i % R.NACC;
-        const uint32_t bph = (uint32_t)(i / R.NACC) & 1u;
-        const float ws = ws_next;
-        if (i + 1 < n) ws_next = wscale_of(my[i + 1]);  // one tile ahead
+        const int s = i % R.S, buf = i % R.nacc;
+        const float w0 = w0n, w1 = w1n;
+        if (i + 1 < n) wscales(my[i + 1], w0n, w1n);  // one tile ahead
         if (e.flags & kSegStart) {
 #pragma unroll
-            for (int b = 0; b < BP; ++b) acc[b] = 0.f;
+            for (int k = 0; k < 64; ++k) acc[k] = 0.f;
         }
-        if (et == 0 && e.mat == 3 && (i == 0 || my[i - 1].mat != 3)) KDA_TR(P, TR_QKV_DONE);
-        if (!dead && !warp_wait_bar(&R.accfull[buf], bph, c, 8)) dead = true;
+        if (threadIdx.x == 128 && e.mat == 3 && (i == 0 || my[i - 1].mat != 3)) KDA_TR(P, TR_QKV_DONE);
+        if (!dead && !warp_wait_bar(&R.mmad[s], (uint32_t)(i / R.S) & 1u, c, 8)) dead = true;
         if (!dead) {
             tc_fence_after();
-            const uint32_t taddr = taddr_base + (uint32_t)(buf * 4 * BP);
-            if (e.mat < 3) accumulate_tile<2, BP>(taddr, R, s, ws, acc);
-            else accumulate_tile<4, BP>(taddr, R, s, ws, acc);
-            mbar_arrive(&R.empty[s]);  // the stage's scales are read
+            const uint32_t tb = tq + (uint32_t)(buf * R.cols);
+            if (e.mat < 3) epi_accumulate<G.gx, G.nx, false>(tb, q, t, R.a(s), G.rsx, w0, w1, acc);
+            else epi_accumulate<G.go, G.no, true>(tb, q, t, R.a(s), G.rso, w0, w1, acc);
             tc_fence_before();
-            mbar_arrive(&R.accempty[buf]);
-            if (et == 0 && i < 32) KDA_TR(P, TR_TILE_EPI + i);
+            __syncwarp();
+            if (t == 0) {
+                mbar_arrive(&R.empty[s]);       // the stage's scales are read, the MMA is done
+                mbar_arrive(&R.accempty[buf]);  // the accumulator is read
+            }
+            if (threadIdx.x == 128 && i < 32) KDA_TR(P, TR_TILE_EPI + i);
         }
         if (!(e.flags & kSegEnd)) continue;
         if (!dead) {
-            float *part = P.part + (size_t)e.seg * BP * 128;
-#pragma unroll
-            for (int b = 0; b < BP; ++b)
-                if (b < P.B) part[b * 128 + row] = acc[b];
+            float *slot = P.part + (size_t)e.seg * slot_floats<BP>();
+            if (e.mat < 3) epi_publish<BP, G.gx, G.nx, false>(slot, q, t, P.B, acc);
+            else epi_publish<BP, G.go, G.no, true>(slot, q, t, P.B, acc);
         }
-        named_bar(1, 128);  // all 128 partial rows are stored before the release
-        if (et == 0 && !dead && !*c.sh_abort) red_release_add(P.ctr + P.off_rb + rb_key(P, e.mat, e.rb), 1u);
+        __syncwarp();  // the warp's partial stores come before lane 0's arrival
+        if (t == 0) mbar_arrive(&R.segdone[nseg % kSegBars]);
+        ++nseg;
+    }
+}
+
+// Warp 3, lane 0: in tile order, each segment's partials are released to the consumers once
+// the four epilogue warps have stored them (the release fence runs here, off the epilogue).
+__device__ void publisher(const FusedParams &P, const Ring &R, const TileEntry *my, int n, const Ctl &c)
+{
+    int k = 0;
+    for (int i = 0; i < n; ++i) {
+        const TileEntry e = my[i];
+        if (!(e.flags & kSegEnd)) continue;
+        const bool ok = wait_bar(&R.segdone[k % kSegBars], (uint32_t)(k / kSegBars) & 1u, c, 9);
+        ++k;
+        if (!ok) break;
+        if (!*c.sh_abort) red_release_add(P.ctr + P.off_rb + rg_key(P, e.mat, e.rg), 1u);
+        if (k - 1 < 7) KDA_TR(P, TR_PUB0 + k - 1);
     }
 }
 
@@ -882,17 +1116,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     Ring R;
     R.S = P.stages;
-    R.sbytes = P.stage_bytes;
-    R.NACC = P.nacc;
-    R.base = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)P.stages * P.stage_bytes);
+    R.a_bytes = P.a_bytes;
+    R.w_bytes = P.w_bytes;
+    R.nacc = P.nacc;
+    R.cols = P.cols;
+    R.a0 = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)P.stages * (P.a_bytes + P.w_bytes));
     R.full = bars;
-    R.empty = bars + kMaxStages;
-    R.accfull = bars + 2 * kMaxStages;
-    R.accempty = bars + 2 * kMaxStages + kMaxAcc;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kMaxStages + 2 * kMaxAcc);
+    R.mmad = bars + kMaxStages;
+    R.empty = bars + 2 * kMaxStages;
+    R.accempty = bars + 3 * kMaxStages;
+    R.segdone = bars + 3 * kMaxStages + kMaxAcc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kMaxStages + kMaxAcc + kSegBars);
     volatile int *sh_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    VecSmem *vs = reinterpret_cast<VecSmem *>(bars + 2 * kMaxStages + 2 * kMaxAcc + 2);
+    VecSmem *vs = reinterpret_cast<VecSmem *>(bars + 3 * kMaxStages + kMaxAcc + kSegBars + 2);
     TileEntry *stiles = reinterpret_cast<TileEntry *>(reinterpret_cast<uint8_t *>(vs) + sizeof(VecSmem));
 
     // this CTA's tile list -> shared memory (read by every role, once per tile)
@@ -903,19 +1140,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < P.stages; ++s) {
-            mbar_init(&R.full[s], 2);          // weight copy + activation copy
-            mbar_init(&R.empty[s], 1 + 128);   // MMA commit + the epilogue's 128 threads
+            mbar_init(&R.full[s], 2);           // weight copy + activation copy
+            mbar_init(&R.mmad[s], 1);           // the tile's MMA commit
+            mbar_init(&R.empty[s], kEpiWarps);  // the epilogue warps are done with the stage
         }
-        for (int b = 0; b < P.nacc; ++b) {
-            mbar_init(&R.accfull[b], 1);
-            mbar_init(&R.accempty[b], 128);
-        }
+        for (int b = 0; b < P.nacc; ++b) mbar_init(&R.accempty[b], kEpiWarps);
+        for (int b = 0; b < kSegBars; ++b) mbar_init(&R.segdone[b], kEpiWarps);
+        for (int b = 0; b < kOHand; ++b) mbar_init(&vs->ohand[b], 1);
+        vs->opub = 0;
         *sh_abort = 0;
         mbar_fence_init();
     }
     if (warp == 3 && lane == 0) {
-        // small inputs every CTA reads soon: pull them into L2 before the weight stream queues up
-        prefetch_l2_slice(P.x, (size_t)P.B * P.H * 2);
+        // small weights every CTA reads soon: pull them into L2 before the weight stream queues up
         prefetch_l2_slice(P.wb, (size_t)P.nh * P.H * 2);
         prefetch_l2_slice(P.wa_down, (size_t)P.r * P.H * 2);
         prefetch_l2_slice(P.wa_up, (size_t)P.nh * P.dk * P.r * 2);
@@ -923,8 +1160,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     if (warp == 0 && lane == 0) {
         for (int m = 0; m < 4; ++m) prefetch_tmap(&P.tm_w[m]);
         prefetch_tmap(&P.tm_xq);
+        prefetch_tmap(&P.tm_xrep);
         prefetch_tmap(&P.tm_oq);
-        if (4 * BP + scale_rows(BP) > 256) prefetch_tmap(&P.tm_osc);
+        prefetch_tmap(&P.tm_orep);
+        if (act_rows(act_geo(BP).go, act_geo(BP).sr) > 256) prefetch_tmap(&P.tm_osc);
     }
     if (warp == 2) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -938,11 +1177,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     const Ctl c{P, sh_abort};
     const TileEntry *my = stiles;
 
+    // Launched with programmatic stream serialization, the next step's grid may start on the
+    // SMs this grid frees.  Before waiting for this grid to finish, it only reads inputs no
+    // kernel writes -- the weights (the first stages of the stream) and its tile lists;
+    // x, the state and every scratch buffer are touched after the wait.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    int pre = 0;
+    if (warp == 0 && lane == 0) pre = preissue_weights<BP>(P, R, my, n);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (warp == 3 && lane == 0) prefetch_l2_slice(P.x, (size_t)P.B * P.H * 2);
+
     if (warp == 0) {
-        if (lane == 0) producer<BP>(P, R, my, n, c);
+        if (lane == 0) producer<BP>(P, R, my, n, c, pre);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) o_publisher(P, vs, c);
+        __syncwarp();
     } else if (warp == 2) {
         if (lane == 0) mma_issuer<BP>(P, R, my, n, tmem, c);
-    } else if (warp >= 4 && warp < 8) {
+        __syncwarp();
+    } else if (warp == 3) {
+        if (lane == 0) publisher(P, R, my, n, c);
+        __syncwarp();
+    } else if (warp >= 4 && warp < 4 + kEpiWarps) {
         epilogue_role<BP>(P, R, my, n, tmem, c);
         if (threadIdx.x == 128) KDA_TR(P, TR_EPI_DONE);
     } else if (warp >= 8) {
@@ -951,7 +1208,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     tc_fence_before();
     __syncthreads();
     if (warp == 2) {
-        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -980,7 +1236,8 @@ PFN_encodeTiled get_encode()
     return fn;
 }
 
-// uint8 matrix [rows, cols] (row-major), box [box_rows, 128 bytes], 128-byte swizzle.
+// uint8 matrix [rows, cols] (row-major), box [box_rows, 128 bytes], 128-byte swizzle.  Rows
+// of a box past the matrix read as zero.
 bool encode_u8_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
 {
     PFN_encodeTiled enc = get_encode();
@@ -1000,16 +1257,34 @@ int bp_for(int B)
     while (bp < B) bp *= 2;
     return bp;
 }
+int class_of(int BP) { return BP <= 8 ? 0 : BP <= 16 ? 1 : BP <= 32 ? 2 : 3; }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// ring stage: weight tile, then up to four activation planes of BP rows and the scale rows
-size_t stage_bytes_for(int BP) { return align_up((size_t)kTileBytes + (4 * BP + scale_rows(BP)) * 128, 1024); }
-
-size_t ctr_words(const Dims &d)
+// shared-memory regions of one ring stage: activation tile, weight tile
+size_t a_bytes_for(int BP)
 {
-    return C_FIXED + (size_t)d.Dv() / 128 + 2 * (d.Dk() / 128) + d.Dv() / 128 + d.H / 128 + 16;
+    const ActGeo g = act_geo(BP);
+    return align_up((size_t)std::max(act_rows(g.gx, g.sr), act_rows(g.go, g.sr)) * 128, 1024);
 }
+size_t w_bytes_for(int BP)
+{
+    const ActGeo g = act_geo(BP);
+    return (size_t)std::max(g.nx, g.no) * 128;
+}
+size_t stage_bytes_for(int BP) { return a_bytes_for(BP) + w_bytes_for(BP); }
+int tmem_cols_for(int BP)
+{
+    const ActGeo g = act_geo(BP);
+    return std::max(g.mhx * g.nx, g.mho * g.no);
+}
+
+int row_group_keys(const Dims &d, const SchedGeo &g)
+{
+    return 2 * ((d.Dk() + g.nx - 1) / g.nx) + (d.Dv() + g.nx - 1) / g.nx + (d.H + g.no - 1) / g.no;
+}
+
+size_t ctr_words(const Dims &d, int max_keys) { return C_FIXED + (size_t)d.Dv() / 128 + max_keys + 16; }
 
 template <int BP, int DK>
 void *kernel_ptr() { return reinterpret_cast<void *>(&k_fused<BP, DK>); }
@@ -1027,6 +1302,37 @@ void *pick_kernel(int BP, int DK)
     case 64128: return kernel_ptr<64, 128>();
     default: return nullptr;
     }
+}
+
+size_t fixed_smem_bytes(int max_tiles)
+{
+    return 1024 /*alignment slack*/ + (3 * kMaxStages + kMaxAcc + kSegBars + 2) * 8 + sizeof(VecSmem) +
+           (size_t)max_tiles * sizeof(TileEntry);
+}
+
+constexpr size_t kSmemBudget = 227 * 1024;
+
+// Schedules of every padded-batch class up to bpm; false if one does not fit the kernel.
+struct ClassPlan {
+    std::vector<TileEntry> tiles;
+    std::vector<uint32_t> off, rbinfo;
+    size_t nseg = 0;
+    int max_tiles = 0, keys = 0;
+};
+bool plan_classes(const Dims &dmax, int num_ctas, int bpm, std::vector<ClassPlan> *plans)
+{
+    plans->clear();
+    for (int BP = 8; BP <= bpm; BP *= 2) {
+        ClassPlan cp;
+        const SchedGeo g = fused_sched_geo(dmax, BP);
+        fused_build_schedule(dmax, num_ctas, g, &cp.tiles, &cp.off, &cp.nseg, &cp.rbinfo);
+        for (int c = 0; c < num_ctas; ++c) cp.max_tiles = std::max(cp.max_tiles, (int)(cp.off[c + 1] - cp.off[c]));
+        if (cp.max_tiles > kMaxTilesPerCta) return false;
+        if (fixed_smem_bytes(cp.max_tiles) + 2 * stage_bytes_for(BP) > kSmemBudget) return false;
+        cp.keys = row_group_keys(dmax, g);
+        plans->push_back(std::move(cp));
+    }
+    return true;
 }
 
 }  // namespace
@@ -1047,20 +1353,24 @@ size_t fused_scratch_bytes(const Dims &dmax, int num_sms)
 {
     if (!fused_supports(Dims{std::min(dmax.B, kMaxBP), dmax.H, dmax.nh, dmax.dk, dmax.dv, dmax.r}, num_sms)) return 0;
     const int bpm = bp_for(std::min(dmax.B, kMaxBP));
-    std::vector<TileEntry> t;
-    std::vector<uint32_t> o;
-    size_t nseg = 0;
-    fused_build_schedule(dmax, num_ctas_for(num_sms), &t, &o, &nseg, nullptr);
-    for (size_t c = 0; c + 1 < o.size(); ++c)
-        if (o[c + 1] - o[c] > (uint32_t)kMaxTilesPerCta) return 0;  // too many tiles per CTA: simple engine
+    std::vector<ClassPlan> plans;
+    if (!plan_classes(dmax, num_ctas_for(num_sms), bpm, &plans)) return 0;  // too many tiles: simple engine
+    const ActGeo g = act_geo(bpm);
+    size_t part = 0, sched = 0;
+    int keys = 0;
+    for (size_t ci = 0; ci < plans.size(); ++ci) {
+        const int BP = 8 << ci;
+        part = std::max(part, plans[ci].nseg * (size_t)2 * BP * 256 * 4);
+        sched += align_up(plans[ci].tiles.size() * sizeof(TileEntry), 256) + align_up(plans[ci].off.size() * 4, 256) +
+                 align_up(plans[ci].rbinfo.size() * 4, 256);
+        keys = std::max(keys, plans[ci].keys);
+    }
     size_t n = 0;
-    n += align_up((size_t)(2 * bpm + scale_rows(bpm)) * dmax.H, 1024);    // x planes + scale rows
-    n += align_up((size_t)(4 * bpm + scale_rows(bpm)) * dmax.Dv(), 1024);  // o planes + scale rows
-    n += align_up(nseg * bpm * 128 * 4, 256);                             // partial sums
-    n += align_up(ctr_words(dmax) * 4, 256);                              // counters
-    n += align_up(t.size() * sizeof(TileEntry), 256);                     // tile lists
-    n += align_up(o.size() * 4, 256);
-    n += align_up((size_t)2 * (2 * (dmax.Dk() / 128) + 2 * (dmax.Dv() / 128) + dmax.H / 128) * 4, 256);  // rbinfo
+    n += align_up((size_t)act_rows(g.gx, g.sr) * dmax.H, 1024);     // x planes + scale rows
+    n += align_up((size_t)act_rows(g.go, g.sr) * dmax.Dv(), 1024);  // o planes + scale rows
+    n += align_up(part, 256);                                // partial sums
+    n += align_up(ctr_words(dmax, keys) * 4, 256);           // counters
+    n += sched;                                              // tile lists, offsets, row-group info
     return n + 1024;
 }
 
@@ -1072,21 +1382,34 @@ void fused_bind_scratch(const Dims &dmax, int num_sms, void *base, size_t bytes,
     const int bpm = bp_for(std::min(dmax.B, kMaxBP));
     fs->bp_max = bpm;
     fs->num_ctas = num_ctas_for(num_sms);
-    fused_build_schedule(dmax, fs->num_ctas, &fs->h_tiles, &fs->h_off, &fs->nseg_total, &fs->h_rbinfo);
-    fs->ntiles = fs->h_tiles.size();
-    fs->max_tiles_per_cta = 0;
-    for (int c = 0; c < fs->num_ctas; ++c)
-        fs->max_tiles_per_cta = std::max(fs->max_tiles_per_cta, (int)(fs->h_off[c + 1] - fs->h_off[c]));
+    std::vector<ClassPlan> plans;
+    plan_classes(dmax, fs->num_ctas, bpm, &plans);
+    fs->nclass = (int)plans.size();
+    const ActGeo g = act_geo(bpm);
+    size_t part = 0;
+    int keys = 0;
+    for (int ci = 0; ci < fs->nclass; ++ci) {
+        const int BP = 8 << ci;
+        part = std::max(part, plans[ci].nseg * (size_t)2 * BP * 256 * 4);
+        keys = std::max(keys, plans[ci].keys);
+        fs->max_tiles_per_cta[ci] = plans[ci].max_tiles;
+        fs->nseg_total = std::max(fs->nseg_total, plans[ci].nseg);
+        fs->h_tiles[ci] = std::move(plans[ci].tiles);
+        fs->h_off[ci] = std::move(plans[ci].off);
+        fs->h_rbinfo[ci] = std::move(plans[ci].rbinfo);
+    }
     char *p = reinterpret_cast<char *>(align_up(reinterpret_cast<uintptr_t>(base), 1024));
     auto take = [&](size_t n, size_t a) { char *r = p; p += align_up(n, a); return r; };
-    fs->xq = (uint8_t *)take((size_t)(2 * bpm + scale_rows(bpm)) * dmax.H, 1024);
-    fs->oq = (uint8_t *)take((size_t)(4 * bpm + scale_rows(bpm)) * dmax.Dv(), 1024);
-    fs->part = (float *)take(fs->nseg_total * bpm * 128 * 4, 256);
-    fs->ctr_bytes = ctr_words(dmax) * 4;
+    fs->xq = (uint8_t *)take((size_t)act_rows(g.gx, g.sr) * dmax.H, 1024);
+    fs->oq = (uint8_t *)take((size_t)act_rows(g.go, g.sr) * dmax.Dv(), 1024);
+    fs->part = (float *)take(part, 256);
+    fs->ctr_bytes = ctr_words(dmax, keys) * 4;
     fs->ctr = (uint32_t *)take(fs->ctr_bytes, 256);
-    fs->tiles = (TileEntry *)take(fs->h_tiles.size() * sizeof(TileEntry), 256);
-    fs->cta_off = (uint32_t *)take(fs->h_off.size() * 4, 256);
-    fs->rbinfo = (uint32_t *)take(fs->h_rbinfo.size() * 4, 256);
+    for (int ci = 0; ci < fs->nclass; ++ci) {
+        fs->tiles[ci] = (TileEntry *)take(fs->h_tiles[ci].size() * sizeof(TileEntry), 256);
+        fs->cta_off[ci] = (uint32_t *)take(fs->h_off[ci].size() * 4, 256);
+        fs->rbinfo[ci] = (uint32_t *)take(fs->h_rbinfo[ci].size() * 4, 256);
+    }
     fs->off_oready = C_FIXED;
     fs->off_rb = fs->off_oready + dmax.Dv() / 128;
 }
@@ -1100,12 +1423,18 @@ cudaError_t fused_init(const Dims &, FusedState *fs)
     }
     if (const char *e = getenv("KDA_DEBUG_SKIP_GATE_RELEASE")) fs->debug_skip_gate_release = atoi(e) != 0;
     if (const char *e = getenv("KDA_STAGES")) fs->stages_override = atoi(e);
-    cudaError_t err = cudaMemcpy(fs->tiles, fs->h_tiles.data(), fs->h_tiles.size() * sizeof(TileEntry),
-                                 cudaMemcpyHostToDevice);
-    if (err == cudaSuccess)
-        err = cudaMemcpy(fs->cta_off, fs->h_off.data(), fs->h_off.size() * 4, cudaMemcpyHostToDevice);
-    if (err == cudaSuccess)
-        err = cudaMemcpy(fs->rbinfo, fs->h_rbinfo.data(), fs->h_rbinfo.size() * 4, cudaMemcpyHostToDevice);
+    fs->early_tiles = kEarlyTilesDefault;
+    if (const char *e = getenv("KDA_EARLY_TILES")) fs->early_tiles = std::max(0, atoi(e));
+    cudaError_t err = cudaGetDevice(&fs->device);
+    for (int ci = 0; ci < fs->nclass && err == cudaSuccess; ++ci) {
+        err = cudaMemcpy(fs->tiles[ci], fs->h_tiles[ci].data(), fs->h_tiles[ci].size() * sizeof(TileEntry),
+                         cudaMemcpyHostToDevice);
+        if (err == cudaSuccess)
+            err = cudaMemcpy(fs->cta_off[ci], fs->h_off[ci].data(), fs->h_off[ci].size() * 4, cudaMemcpyHostToDevice);
+        if (err == cudaSuccess)
+            err = cudaMemcpy(fs->rbinfo[ci], fs->h_rbinfo[ci].data(), fs->h_rbinfo[ci].size() * 4,
+                             cudaMemcpyHostToDevice);
+    }
 #ifdef KDA_TRACE
     if (err == cudaSuccess) err = cudaMalloc(&fs->trace, (size_t)fs->num_ctas * kTraceSlots * 8);
     if (err == cudaSuccess) err = cudaMemset(fs->trace, 0, (size_t)fs->num_ctas * kTraceSlots * 8);
@@ -1126,9 +1455,12 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
                        FusedState &fs, const Scratch &s, int *status, cudaStream_t stream)
 {
     if (!fs.uploaded) return cudaErrorNotReady;
-    const int BP = bp_for(d.B);
+    const int BP = bp_for(d.B), cls = class_of(BP);
     void *kern = pick_kernel(BP, d.dk);
-    if (!kern || BP > fs.bp_max) return cudaErrorNotSupported;
+    if (!kern || cls >= fs.nclass) return cudaErrorNotSupported;
+    const ActGeo g = act_geo(BP);
+    const SchedGeo sg = fused_sched_geo(d, BP);
+    if (fs.last_class >= 0 && fs.last_class != cls) fs.needs_reset = true;  // row-group counters differ per class
     if (fs.needs_reset) {
         cudaError_t e = cudaMemsetAsync(fs.ctr, 0, fs.ctr_bytes, stream);
         if (e != cudaSuccess) return e;
@@ -1138,13 +1470,15 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     }
     static thread_local FusedParams P;
     memset(&P, 0, sizeof P);
-    // weight maps (cached by pointer)
+    // weight maps (cached by pointer and tile rows)
     const void *keys[4] = {w.wq, w.wk, w.wv, w.wo};
+    const int box[4] = {g.nx, g.nx, g.nx, g.no};
     int slot = -1;
-    for (int i = 0; i < 4 && slot < 0; ++i)
-        if (fs.map_keys[i][0] == keys[0] && fs.map_keys[i][1] == keys[1] && fs.map_keys[i][2] == keys[2] &&
-            fs.map_keys[i][3] == keys[3])
-            slot = i;
+    for (int i = 0; i < 4 && slot < 0; ++i) {
+        bool hit = true;
+        for (int m = 0; m < 4; ++m) hit = hit && fs.map_keys[i][m] == keys[m] && fs.map_box[i][m] == box[m];
+        if (hit) slot = i;
+    }
     if (slot < 0) {
         slot = fs.map_next;
         fs.map_next = (fs.map_next + 1) & 3;
@@ -1152,19 +1486,33 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
         const uint64_t cols[4] = {(uint64_t)d.H, (uint64_t)d.H, (uint64_t)d.H, (uint64_t)d.Dv()};
         for (int m = 0; m < 4; ++m) {
             fs.map_keys[slot][m] = nullptr;
-            if (!encode_u8_map(&fs.wmaps[slot][m], keys[m], rows[m], cols[m], 128)) return cudaErrorInvalidValue;
+            if (!encode_u8_map(&fs.wmaps[slot][m], keys[m], rows[m], cols[m], (uint32_t)box[m]))
+                return cudaErrorInvalidValue;
         }
-        for (int m = 0; m < 4; ++m) fs.map_keys[slot][m] = keys[m];
+        for (int m = 0; m < 4; ++m) {
+            fs.map_keys[slot][m] = keys[m];
+            fs.map_box[slot][m] = box[m];
+        }
     }
     for (int m = 0; m < 4; ++m) P.tm_w[m] = fs.wmaps[slot][m];
-    const int sr = scale_rows(BP);
-    if (!encode_u8_map(&P.tm_xq, fs.xq, 2 * BP + sr, d.H, 2 * BP + sr)) return cudaErrorInvalidValue;
-    if (4 * BP + sr <= 256) {
-        if (!encode_u8_map(&P.tm_oq, fs.oq, 4 * BP + sr, d.Dv(), 4 * BP + sr)) return cudaErrorInvalidValue;
-    } else {
-        if (!encode_u8_map(&P.tm_oq, fs.oq, 4 * BP + sr, d.Dv(), 4 * BP)) return cudaErrorInvalidValue;
-        if (!encode_u8_map(&P.tm_osc, fs.oq, 4 * BP + sr, d.Dv(), sr)) return cudaErrorInvalidValue;
+    // activation-plane maps (fixed per handle and class): x tile and one x group; o tile, its
+    // scale rows past 256 and one o group
+    if (!fs.amap_ok[cls]) {
+        const ActGeo gm = act_geo(fs.bp_max);  // buffer rows are sized for the largest class
+        const int xrows = act_rows(gm.gx, gm.sr), orows = act_rows(gm.go, gm.sr), ro = act_rows(g.go, g.sr);
+        if (!encode_u8_map(&fs.amaps[cls][0], fs.xq, xrows, d.H, act_main_rows(g.gx, g.sr)) ||
+            !encode_u8_map(&fs.amaps[cls][1], fs.xq, xrows, d.H, 16) ||
+            !encode_u8_map(&fs.amaps[cls][2], fs.oq, orows, d.Dv(), act_main_rows(g.go, g.sr)) ||
+            !encode_u8_map(&fs.amaps[cls][3], fs.oq, orows, d.Dv(), ro > 256 ? ro - 256 : 16) ||
+            !encode_u8_map(&fs.amaps[cls][4], fs.oq, orows, d.Dv(), 16))
+            return cudaErrorInvalidValue;
+        fs.amap_ok[cls] = true;
     }
+    P.tm_xq = fs.amaps[cls][0];
+    P.tm_xrep = fs.amaps[cls][1];
+    P.tm_oq = fs.amaps[cls][2];
+    P.tm_osc = fs.amaps[cls][3];
+    P.tm_orep = fs.amaps[cls][4];
     P.wscale[0] = w.sq;
     P.wscale[1] = w.sk;
     P.wscale[2] = w.sv;
@@ -1185,8 +1533,8 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.t = s.t;
     P.ctr = fs.ctr;
     P.trace = fs.trace;
-    P.tiles = fs.tiles;
-    P.cta_off = fs.cta_off;
+    P.tiles = fs.tiles[cls];
+    P.cta_off = fs.cta_off[cls];
     P.status = status;
     P.B = d.B;
     P.H = d.H;
@@ -1196,41 +1544,46 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.r = d.r;
     P.nKBx = d.H / 128;
     P.nKBo = d.Dv() / 128;
-    P.nRBq = d.Dk() / 128;
-    P.nRBv = d.Dv() / 128;
+    P.nRGq = (d.Dk() + sg.nx - 1) / sg.nx;
+    P.nRGv = (d.Dv() + sg.nx - 1) / sg.nx;
+    P.nRGo = (d.H + sg.no - 1) / sg.no;
     P.off_oready = fs.off_oready;
     P.off_rb = fs.off_rb;
-    P.rbinfo = reinterpret_cast<const uint2 *>(fs.rbinfo);
-    P.nRBo = d.H / 128;
+    P.rbinfo = reinterpret_cast<const uint2 *>(fs.rbinfo[cls]);
     const uint32_t epoch = fs.epoch + 1;
     P.epoch = epoch;
     P.t_xq = (fs.cum_b + (uint32_t)d.B) * (uint32_t)P.nKBx;
+    P.early_tiles = fs.early_tiles;
     P.t_gate = epoch * (uint32_t)(d.nh + d.r);
     P.t_o = fs.cum_b + (uint32_t)d.B;
     P.timeout_ns = fs.timeout_ns;
     P.out_bf16 = out_dtype == KDA_OUT_BF16;
     P.skip_gate_release = fs.debug_skip_gate_release;
+    P.a_bytes = (int)a_bytes_for(BP);
+    P.w_bytes = (int)w_bytes_for(BP);
+    P.cols = tmem_cols_for(BP);
+    P.nacc = std::min(kMaxAcc, kTmemCols / P.cols);
     const size_t sbytes = stage_bytes_for(BP);
-    P.nacc = std::min(kMaxAcc, kTmemCols / (4 * BP));
-    const size_t fixed = 1024 /*alignment slack*/ + (2 * kMaxStages + 2 * kMaxAcc + 2) * 8 + sizeof(VecSmem) +
-                         (size_t)fs.max_tiles_per_cta * sizeof(TileEntry);
-    const size_t budget = 227 * 1024;
-    if (fixed + 2 * sbytes > budget) return cudaErrorNotSupported;
-    int stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / sbytes);
-    if (fs.stages_override > 0) stages = std::min(stages, std::max(2, fs.stages_override));
+    const size_t fixed = fixed_smem_bytes(fs.max_tiles_per_cta[cls]);
+    if (fixed + 2 * sbytes > kSmemBudget) return cudaErrorNotSupported;
+    int stages = (int)std::min<size_t>(kMaxStagesDefault, (kSmemBudget - fixed) / sbytes);
+    if (fs.stages_override > 0)
+        stages = (int)std::min<size_t>({(size_t)kMaxStages, (kSmemBudget - fixed) / sbytes,
+                                        (size_t)std::max(2, fs.stages_override)});
     P.stages = stages;
-    P.stage_bytes = (int)sbytes;
     const size_t smem = (size_t)stages * sbytes + fixed;
 
+    // the dynamic shared-memory limit is a per-device attribute of the kernel
     static std::mutex mu;
-    static std::map<void *, size_t> configured;
+    static std::map<std::pair<int, void *>, size_t> configured;
     {
         std::lock_guard<std::mutex> lk(mu);
-        auto it = configured.find(kern);
+        const auto key = std::make_pair(fs.device, kern);
+        auto it = configured.find(key);
         if (it == configured.end() || it->second < smem) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
-            configured[kern] = smem;
+            configured[key] = smem;
         }
     }
     cudaLaunchConfig_t cfg = {};
@@ -1238,14 +1591,23 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    // Every CTA must be resident at once (they wait on one another, with bounded waits): one
+    // CTA per SM and a grid of one CTA per SM.  A cooperative launch makes the runtime check
+    // that; with launch overlap the grid instead starts on the SMs the previous step frees.
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    if (fs.overlap) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void *args[1] = {&P};
     cudaError_t e = cudaLaunchKernelExC(&cfg, kern, args);
     if (e != cudaSuccess) return e;
+    fs.last_class = cls;
     fs.epoch = epoch;
     fs.cum_b += (uint32_t)d.B;
     return cudaSuccess;

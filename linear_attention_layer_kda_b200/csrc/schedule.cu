@@ -9,77 +9,80 @@
 #include "fused.cuh"
 
 namespace kda {
-namespace {
 
-constexpr int kHeadsPerGroup = 8;
-// Head groups of q/k/v tiles between a group's q/k/v tiles and its W_o tiles (-1: all W_o
-// tiles after all q/k/v tiles).  Measured at batch 8: interleaving (1, 2, 3) stalls the MMA on
-// o blocks whose state units are still running, so the default keeps W_o last.
-constexpr int kWoLag = -1;
-
-}  // namespace
-
-// Tile order and segments.  Heads are taken in groups of eight; group g contributes the
-// q, k and v row blocks of its heads (all K blocks), split into contiguous equal runs over
-// the CTAs; then the W_o tiles whose K blocks belong to group g, split the same way.  A
-// segment is a CTA's run inside one row block; its partial-sum slot is numbered row block
-// by row block so the segments of a row block are adjacent.
-void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, std::vector<uint32_t> *off,
-                          size_t *nseg_total, std::vector<uint32_t> *rbinfo)
+// Row groups of N = 256 weight rows while the epilogue's running sums allow it (fewer for
+// 32 and 64 sequences); runs of BP / 2 tiles (4 at most batch sizes) so that the partial sums
+// a run writes stay a small fraction of the weight bytes it streams.
+SchedGeo fused_sched_geo(const Dims &dmax, int BP)
 {
-    const int nKBx = d.H / 128, nKBo = d.Dv() / 128, nRBq = d.Dk() / 128, nRBv = d.Dv() / 128, nRBo = d.H / 128;
-    const int hpu = std::max(128 / d.dk, 128 / d.dv);
-    int heads_per_group = kHeadsPerGroup, wo_lag = kWoLag;
-    if (const char *e = getenv("KDA_HEADS_PER_GROUP")) heads_per_group = std::max(1, atoi(e));
-    if (const char *e = getenv("KDA_WO_LAG")) wo_lag = atoi(e);
-    const int hpg = std::max(hpu, heads_per_group / hpu * hpu);
-    const int G = (d.nh + hpg - 1) / hpg;
-    struct T { uint8_t mat; uint16_t rb, kb; };
-    std::vector<std::vector<T>> per_cta(P);
-    // Contiguous runs in CTA order; the n % P longer runs go to the CTAs with the fewest
-    // tiles so far, so that the totals over all groups differ by at most one tile.
-    auto split = [&](const std::vector<T> &list) {
-        const size_t n = list.size(), base = n / P, extra = n % P;
-        std::vector<int> order(P);
-        for (int c = 0; c < P; ++c) order[c] = c;
-        std::stable_sort(order.begin(), order.end(),
-                         [&](int a, int b) { return per_cta[a].size() < per_cta[b].size(); });
-        std::vector<size_t> len(P, base);
-        for (size_t j = 0; j < extra; ++j) len[order[j]]++;
-        size_t pos = 0;
-        for (int c = 0; c < P; ++c)
-            for (size_t i = 0; i < len[c]; ++i) per_cta[c].push_back(list[pos++]);
-    };
-    auto qkv_group = [&](int g) {
-        const int h0 = g * hpg, h1 = std::min(d.nh, h0 + hpg);
-        std::vector<T> list;
-        for (int m = 0; m < 3; ++m) {
-            const int hd = m == 2 ? d.dv : d.dk;
-            for (int rb = h0 * hd / 128; rb < h1 * hd / 128; ++rb)
-                for (int kb = 0; kb < nKBx; ++kb) list.push_back(T{(uint8_t)m, (uint16_t)rb, (uint16_t)kb});
-        }
-        split(list);
-    };
-    auto wo_group = [&](int g) {
-        const int h0 = g * hpg, h1 = std::min(d.nh, h0 + hpg);
-        std::vector<T> list;
-        for (int rb = 0; rb < nRBo; ++rb)
-            for (int kb = h0 * d.dv / 128; kb < h1 * d.dv / 128; ++kb) list.push_back(T{3, (uint16_t)rb, (uint16_t)kb});
-        split(list);
-    };
-    // The W_o tiles of group g follow the q/k/v tiles of group g + lag, so the state units of
-    // group g run while the weight stream carries later groups' q/k/v.
-    const int lag = wo_lag < 0 ? G : wo_lag;
-    for (int g = 0; g < G; ++g) {
-        qkv_group(g);
-        if (g - lag >= 0) wo_group(g - lag);
+    const ActGeo g = act_geo(BP);
+    const int nkb = dmax.H / 128;
+    return SchedGeo{g.nx, g.no, std::max(1, std::min(nkb, std::max(4, BP / 2)))};
+}
+
+// Tile order and segments.
+//
+// A tile is `rows` weight rows (a row group) x one 128-wide K block.  The q, k and v row
+// groups are listed in the order of the first head they hold (q, k, v of the same heads side
+// by side), each with all its K blocks; then the W_o tiles, in chunks of `run` consecutive K
+// blocks (o blocks, i.e. heads): chunk 0 for every output row group, then chunk 1, ...
+//
+// The list is dealt out in waves: wave w gives CTA c the `run` tiles at list positions
+// (w * P + c) * run ..., so all SMs stream the earliest heads' weights first and those heads'
+// q/k/v are final long before the stream ends; the state units of early heads, and the W_o
+// tiles that read their o blocks, then overlap the rest of the stream.  The tiles left over
+// after the last full wave are split into P contiguous pieces of equal size (+-1), so every
+// CTA streams the same number of tiles to within one.
+//
+// A segment is a CTA's run of consecutive tiles of one row group; its partial sum goes to its
+// own slot.  Slots are numbered row group by row group, so the slots of a row group are
+// adjacent (rbinfo: first slot, count).
+void fused_build_schedule(const Dims &d, int P, const SchedGeo &g, std::vector<TileEntry> *tiles,
+                          std::vector<uint32_t> *off, size_t *nseg_total, std::vector<uint32_t> *rbinfo)
+{
+    const int nKBx = d.H / 128, nKBo = d.Dv() / 128;
+    const int nRGq = (d.Dk() + g.nx - 1) / g.nx, nRGv = (d.Dv() + g.nx - 1) / g.nx, nRGo = (d.H + g.no - 1) / g.no;
+    int run = std::max(1, g.run);
+    if (const char *e = getenv("KDA_RUN")) run = std::max(1, atoi(e));
+    struct T { uint8_t mat; uint16_t rg, kb; };
+    std::vector<T> list;
+    list.reserve((size_t)(2 * nRGq + nRGv) * nKBx + (size_t)nRGo * nKBo);
+    // q/k/v row groups by first head, then matrix
+    struct G { int head, mat, rg; };
+    std::vector<G> groups;
+    for (int rg = 0; rg < nRGq; ++rg) {
+        groups.push_back(G{rg * g.nx / d.dk, 0, rg});
+        groups.push_back(G{rg * g.nx / d.dk, 1, rg});
     }
-    for (int g = std::max(0, G - lag); g < G; ++g) wo_group(g);
-    // row-block keys: q 0.., k nRBq.., v 2nRBq.., o 2nRBq+nRBv..
+    for (int rg = 0; rg < nRGv; ++rg) groups.push_back(G{rg * g.nx / d.dv, 2, rg});
+    std::stable_sort(groups.begin(), groups.end(),
+                     [](const G &a, const G &b) { return a.head != b.head ? a.head < b.head : a.mat < b.mat; });
+    for (const G &x : groups)
+        for (int kb = 0; kb < nKBx; ++kb) list.push_back(T{(uint8_t)x.mat, (uint16_t)x.rg, (uint16_t)kb});
+    for (int k0 = 0; k0 < nKBo; k0 += run)
+        for (int rg = 0; rg < nRGo; ++rg)
+            for (int kb = k0; kb < std::min(nKBo, k0 + run); ++kb) list.push_back(T{3, (uint16_t)rg, (uint16_t)kb});
+
+    std::vector<std::vector<T>> per_cta(P);
+    const size_t n = list.size();
+    size_t pos = 0;
+    while (n - pos >= (size_t)P * run) {  // full waves
+        for (int c = 0; c < P; ++c)
+            for (int i = 0; i < run; ++i) per_cta[c].push_back(list[pos++]);
+    }
+    {  // the rest, in P contiguous pieces of equal size (+-1)
+        const size_t rest = n - pos, base = rest / P, extra = rest % P;
+        for (int c = 0; c < P; ++c) {
+            const size_t len = base + ((size_t)c < extra ? 1 : 0);
+            for (size_t i = 0; i < len; ++i) per_cta[c].push_back(list[pos++]);
+        }
+    }
+
+    // row-group keys: q 0.., k nRGq.., v 2 nRGq.., o 2 nRGq + nRGv..
     auto key = [&](const T &t) {
-        return t.mat == 3 ? 2 * nRBq + nRBv + t.rb : (t.mat == 2 ? 2 * nRBq + t.rb : t.mat * nRBq + t.rb);
+        return t.mat == 3 ? 2 * nRGq + nRGv + t.rg : (t.mat == 2 ? 2 * nRGq + t.rg : t.mat * nRGq + t.rg);
     };
-    const int nkeys = 2 * nRBq + nRBv + nRBo;
+    const int nkeys = 2 * nRGq + nRGv + nRGo;
     std::vector<uint32_t> nseg(nkeys, 0), seg0(nkeys, 0);
     for (int c = 0; c < P; ++c) {
         const auto &L = per_cta[c];
@@ -102,7 +105,7 @@ void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, s
             const int k = key(L[i]);
             TileEntry e{};
             e.mat = L[i].mat;
-            e.rb = L[i].rb;
+            e.rg = L[i].rg;
             e.kb = L[i].kb;
             const bool start = i == 0 || key(L[i - 1]) != k;
             const bool end = i + 1 == L.size() || key(L[i + 1]) != k;
@@ -123,7 +126,6 @@ void fused_build_schedule(const Dims &d, int P, std::vector<TileEntry> *tiles, s
             (*rbinfo)[2 * k + 1] = nseg[k];
         }
     }
-    (void)nKBo;
 }
 
 }  // namespace kda

@@ -22,8 +22,9 @@ def block_report(got, ref, shape):
 
 
 def run_parity(inp, steps, engine=binding.KDA_ENGINE_AUTO, out_dtype=binding.KDA_OUT_F32, batch=None,
-               max_batch=None, check_every=1):
-    """Runs `steps` steps on both sides; returns a list of (out_err, state_err) per checked step."""
+               max_batch=None, check_every=1, return_state=False):
+    """Runs `steps` steps on both sides; returns a list of (out_err, state_err) per checked step
+    and the engine used (and, with return_state, the CUDA path's final state as fp64)."""
     import torch
     s = inp.shape
     B = s.batch if batch is None else batch
@@ -51,8 +52,11 @@ def run_parity(inp, steps, engine=binding.KDA_ENGINE_AUTO, out_dtype=binding.KDA
                     print(block_report(got_state, S, s))
                 errs.append((t, eo, es))
         dec.sync()
+        final = state.double().cpu().numpy() if return_state else None
     finally:
         engine_used = dec.engine(B)
         dec.close()
         model.close()
+    if return_state:
+        return errs, engine_used, final
     return errs, engine_used

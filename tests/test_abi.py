@@ -141,3 +141,29 @@ def test_header_compiles_as_c99_and_host_calls_behave(lib, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "abi_check ok" in r.stdout
+
+
+def test_noalloc_checks_shape_only(lib):
+    """kda_decode_step_noalloc ignores max_batch and engine: a config with max_batch 0 and an
+    unknown engine passes validation (and then, without a GPU, stops at the device check),
+    while a bad shape or out dtype is still rejected before any CUDA call."""
+    import ctypes
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the call would run")
+    from linear_attention_layer_kda_b200 import binding as b
+    w = b.kda_weights()
+    for n in b.WEIGHT_FIELDS:
+        setattr(w, n, 0x1000)
+    ptr = ctypes.c_void_p
+    x, st, out = ptr(0x100000), ptr(0x200000000), ptr(0x300000000)
+
+    def call(**over):
+        kw = dict(hidden=256, num_heads=2, head_dk=64, head_dv=64, alpha_rank=64, max_batch=0, engine=99)
+        kw.update(over)
+        c = b.make_config(**kw)
+        return lib.kda_decode_step_noalloc(ctypes.byref(c), x, ctypes.byref(w), st, out, 1, None)
+
+    assert call() in (b.KDA_ERR_NO_DEVICE, b.KDA_ERR_CUDA)
+    assert call(hidden=100) == b.KDA_ERR_UNSUPPORTED_SHAPE
+    assert call(out_dtype=5) == b.KDA_ERR_INVALID_ARG

@@ -3,12 +3,15 @@
 Tolerances are the decode benchmark's: max-norm relative error <= 2e-3 on
 out and <= 1e-3 on the updated state, every checked step.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 
 from linear_attention_layer_kda_b200 import binding, inputs as I
 
 from gpu_util import OUT_TOL, STATE_TOL, run_parity
+from helpers import gate_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -97,7 +100,7 @@ def test_replays_are_bitwise_identical():
     s0 = tensors.state_tensor(inp.state0)
     out = torch.empty(8, shape.hidden, device="cuda")
     ref_out = ref_state = None
-    for _ in range(50):
+    for _ in range(1000):
         st = s0.clone()
         dec.step(x, w, st, out)
         dec.sync()
@@ -180,3 +183,57 @@ def test_stage_intermediates_match_oracle(engine):
         blocks = [np.abs(got[:, i:i + 128] - ref[:, i:i + 128]).max() for i in range(0, ref.shape[1], 128)]
         assert err < 1e-4, f"debug tensor {which}: max rel err {err:.3e}; per-block abs err {blocks}"
     dec.close()
+
+
+# ------------------------------------------------------------------ the method's edge cases
+
+def _one_x(inp, steps):
+    """Every step and every sequence sees x row 0 of step 0 (the gate weights below saturate
+    beta or alpha for that one row); the states of the sequences still differ."""
+    x0 = inp.x[0][:1]
+    return dataclasses.replace(inp, x=[np.repeat(x0, inp.shape.batch, axis=0) for _ in range(steps)])
+
+
+def _wide_x(shape, steps):
+    """x whose every 128-wide block mixes magnitudes 2^20 apart (odd positions scaled by
+    2^-20): the small half falls below the two E4M3 planes' floor, 2^-10 of the block scale."""
+    xs = []
+    for t in range(steps):
+        v = I.bf16_bits_to_f64(I.gen_x(shape, t))
+        v[:, 1::2] *= 2.0 ** -20
+        xs.append(I.round_to_bf16_bits(v))
+    return xs
+
+
+EDGE_CASES = ["beta0_alpha1", "alpha0", "wk0", "wide_x"]
+
+
+def _edge_inputs(shape, steps, case):
+    inp = I.generate(shape, steps=steps)
+    if case == "beta0_alpha1":
+        inp = _one_x(inp, steps)
+        wb, wd, wu = gate_weights(shape, inp.x[0][0], beta_mode="zero", alpha_mode="one", base=inp)
+        return dataclasses.replace(inp, wb=wb, wa_down=wd, wa_up=wu)
+    if case == "alpha0":
+        inp = _one_x(inp, steps)
+        _, wd, wu = gate_weights(shape, inp.x[0][0], alpha_mode="zero", base=inp)
+        return dataclasses.replace(inp, wa_down=wd, wa_up=wu)
+    if case == "wk0":
+        return dataclasses.replace(inp, wk=np.zeros_like(inp.wk))
+    return dataclasses.replace(inp, x=_wide_x(shape, steps))
+
+
+@pytest.mark.parametrize("case", EDGE_CASES)
+@pytest.mark.parametrize("engine", ENGINES)
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_edge_cases_match_oracle(cfg, engine, case):
+    """Saturated gates (beta = 0 with alpha = 1; alpha -> 0 at z ~ +3e5), a zero key (W_k = 0,
+    so k^ = 0) and wide-range x blocks, through the CUDA path against the oracle."""
+    shape = I.CONFIGS[cfg]
+    steps = 3 if cfg == 0 else 1
+    inp = _edge_inputs(shape, steps, case)
+    errs, used, final = run_parity(inp, steps, engine=engine, return_state=True)
+    _assert_ok(errs, f"{shape.name} {case}")
+    if case == "beta0_alpha1":  # S' = S: the state must come back unchanged
+        s0 = inp.state0.astype(np.float64)
+        assert np.abs(final - s0).max() <= 1e-6 * np.abs(s0).max()
