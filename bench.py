@@ -49,14 +49,15 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 
-def ideal_bytes(s: I.KdaShape, B: int, out_bytes: int = 4) -> int:
-    """Algorithmic bytes of one step: weights, scales, gate weights, state read + write, x, out."""
+def ideal_bytes(s: I.KdaShape, B: int, out_bytes: int = 4, tokens: int = 1) -> int:
+    """Algorithmic bytes of one step: weights, scales, gate weights, state read + write, x, out
+    (x and out for every token of every sequence; the state is read and written once)."""
     H, Dk, Dv, nh, r = s.hidden, s.dk_total, s.dv_total, s.num_heads, s.alpha_rank
     fp8 = 2 * Dk * H + Dv * H + H * Dv
     scales = 4 * ((Dk // 128) * (H // 128) * 2 + (Dv // 128) * (H // 128) + (H // 128) * (Dv // 128))
     gates = 2 * (r * H + Dk * r + nh * H)
     state = 2 * B * nh * s.head_dk * s.head_dv * 4
-    return fp8 + scales + gates + state + B * H * 2 + B * H * out_bytes
+    return fp8 + scales + gates + state + B * tokens * H * (2 + out_bytes)
 
 
 def ideal_flops(s: I.KdaShape, B: int) -> int:
@@ -259,6 +260,11 @@ def run_reference(args, shape, rank, world):
     return 0
 
 
+def token_rows(xs, T):
+    """x of T consecutive tokens of every sequence as one [B * T, H] array (row b * T + t)."""
+    return np.ascontiguousarray(np.stack(xs[:T], axis=1).reshape(-1, xs[0].shape[1]))
+
+
 def rank_inputs(shape: I.KdaShape, rank: int, world: int):
     """Inputs of one rank: weights shared by all ranks; x and state are this rank's own
     sequences, rows rank*B .. rank*B + B - 1 of the job's counter-based streams, so the N
@@ -312,23 +318,33 @@ def run_ours(args, shape, rank, world, local_rank):
     props = torch.cuda.get_device_properties(dev)
     l2 = max(L2_ASSUMED, int(getattr(props, "L2_cache_size", L2_ASSUMED)))
 
+    TK = args.tokens
+    if TK > 1:
+        shape = shape.replace(steps=max(shape.steps, TK))
     inp = rank_inputs(shape, rank, world)
     T = len(inp.x)  # fresh x per step for multi-step workloads
-    set_bytes = ideal_bytes(shape, B)
+    set_bytes = ideal_bytes(shape, B, tokens=TK)
     R = rotation_sets(shape, l2)
     wts = [tensors.to_device_weights(inp, dev) for _ in range(R)]
     ws = [tensors.weights_struct(w) for w in wts]
     states = [tensors.state_tensor(inp.state0, dev) for _ in range(R)]
-    xs = [tensors.bf16_tensor(inp.x[t], dev) for t in range(T)]
-    outs = [torch.empty(B, shape.hidden, device=dev, dtype=torch.float32) for _ in range(R)]
-    dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, B,
+    if TK > 1:  # one multi-token step: x of T consecutive tokens of every sequence
+        xs = [tensors.bf16_tensor(token_rows(inp.x, TK), dev)]
+        T = 1
+    else:
+        xs = [tensors.bf16_tensor(inp.x[t], dev) for t in range(T)]
+    outs = [torch.empty(B * TK, shape.hidden, device=dev, dtype=torch.float32) for _ in range(R)]
+    dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, B * TK,
                              engine=args.engine)
-    engine = dec.engine(B)
-    launches = dec.launches_per_step(B)
+    engine = dec.engine(B) if TK == 1 else dec.tokens_engine(B, TK)
+    launches = dec.launches_per_step(B) if TK == 1 else (1 if engine == 2 else dec.launches_per_step(B))
 
     def one(i):
         j = i % R
-        dec.step(xs[i % T], ws[j], states[j], outs[j])
+        if TK == 1:
+            dec.step(xs[i % T], ws[j], states[j], outs[j])
+        else:
+            dec.step_tokens(xs[0], ws[j], states[j], outs[j], B, TK)
 
     for i in range(max(3, args.warmup)):
         one(i)
@@ -386,22 +402,25 @@ def run_ours(args, shape, rank, world, local_rank):
 
     # end to end through the host-buffer entry point: H2D x, step, D2H out, sync, every step,
     # on every rank; the slowest rank's wall time sets the job's rate
-    xh = [torch.from_numpy(inp.x[t].view(np.int16)).view(torch.bfloat16).pin_memory() for t in range(T)]
-    oh = torch.empty(B, shape.hidden, dtype=torch.float32).pin_memory()
-    n_e2e = args.e2e_steps if args.e2e_steps > 0 else max(10, min(args.steps, 2000))
-    for i in range(3):
-        dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
-    if world > 1:
-        dist.barrier()
-    t0 = time.perf_counter()
-    for i in range(n_e2e):
-        dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
-    dt = max_over_ranks(time.perf_counter() - t0, world, dev)
-    e2e = {"value": job_steps_per_s(1000.0 * dt / n_e2e, world), "unit": "steps/s",
-           "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 4), "steps": n_e2e}
+    e2e = None
+    if TK == 1:
+        xh = [torch.from_numpy(inp.x[t].view(np.int16)).view(torch.bfloat16).pin_memory() for t in range(T)]
+        oh = torch.empty(B, shape.hidden, dtype=torch.float32).pin_memory()
+        n_e2e = args.e2e_steps if args.e2e_steps > 0 else max(10, min(args.steps, 2000))
+        for i in range(3):
+            dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for i in range(n_e2e):
+            dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
+        dt = max_over_ranks(time.perf_counter() - t0, world, dev)
+        e2e = {"value": job_steps_per_s(1000.0 * dt / n_e2e, world), "unit": "steps/s",
+               "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 4),
+               "steps": n_e2e}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and TK == 1:
         rate, n, cores = oracle_rate(shape, inp, seqs=B, budget_s=args.cpu_seconds, max_steps=1000)
         rate1, n1, _ = oracle_rate(shape, inp, seqs=1, budget_s=min(5.0, args.cpu_seconds), max_steps=50, threads=1)
         cpu = {"value": rate, "unit": "steps/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
@@ -421,7 +440,7 @@ def run_ours(args, shape, rank, world, local_rank):
     hbm_peak = peaks.get("hbm_gbs")
     peak_src = "measured" if hbm_peak else "fallback"
     hbm_peak = float(hbm_peak or FALLBACK_HBM_GBS)
-    ib = ideal_bytes(shape, B)
+    ib = ideal_bytes(shape, B, tokens=TK)
     achieved = ib / (ms_per_step * 1e-3) / 1e9
     traffic = None
     tfile = os.path.join(ROOT, "profiles", f"traffic_{shape.name}.json")
@@ -436,8 +455,8 @@ def run_ours(args, shape, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(shape, world, R),
-        "tokens_per_s": value * B,
+        "config": dict(workload_config(shape, world, R), **({"tokens_per_step": TK} if TK > 1 else {})),
+        "tokens_per_s": value * B * TK,
         "step_us": {"median": med * 1e3, "p10": p10 * 1e3, "p90": p90 * 1e3,
                     "note": "second pass, an event after every step on the launching stream (rank 0); "
                             "the events also stop consecutive steps from overlapping"},
@@ -501,6 +520,8 @@ def parse_args(argv=None):
     ap.add_argument("--clock-window", type=float, default=0.5,
                     help="seconds of untimed steps before the timed region, so clocks settle under load")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the host-buffer end-to-end loop")
+    ap.add_argument("--tokens", type=int, default=1,
+                    help="tokens per sequence in one step (multi-token verify through kda_decode_step_tokens)")
     ap.add_argument("--launch-limit", type=int, default=900, help="seconds before a self-launched job is killed")
     ap.add_argument("--print-rank", action="store_true", help=argparse.SUPPRESS)  # launcher self-check
     return ap.parse_args(argv)

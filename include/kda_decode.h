@@ -160,10 +160,13 @@ KDA_API int kda_decode_step_host(kda_handle h, const void *x_host, const kda_wei
  *   out          [batch * tokens, H] (cfg.out_dtype); row b * tokens + t is the output of
  *                token t, read out after token t's update
  * The projections read the weights once for all batch * tokens rows.  Requires
- * tokens >= 1 and batch * tokens <= max_batch.  tokens == 1 is kda_decode_step; more
- * tokens run the five-kernel engine (KDA_ENGINE_SIMPLE kernels, one state kernel that
- * applies the tokens in order).  The result equals `tokens` successive kda_decode_step
- * calls on that engine bit for bit.  Same errors and ordering as kda_decode_step.
+ * tokens >= 1 and batch * tokens <= max_batch.  tokens == 1 is kda_decode_step.  With up
+ * to 8 tokens and batch * tokens <= 64 rows the fused engine runs the step as one kernel:
+ * each of its state units keeps its sequence's state in registers and applies the tokens in
+ * order.  Otherwise (or with KDA_ENGINE_SIMPLE) the five-kernel engine runs it, with one
+ * state kernel that applies the tokens in order; its result then equals `tokens` successive
+ * kda_decode_step calls on that engine bit for bit.  kda_decode_tokens_engine says which
+ * engine a (batch, tokens) step uses.  Same errors and ordering as kda_decode_step.
  */
 KDA_API int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out,
                                    int batch, int tokens);
@@ -208,6 +211,9 @@ KDA_API int kda_decode_destroy(kda_handle h);
 
 /* Engine the handle runs for `batch` (KDA_ENGINE_SIMPLE or KDA_ENGINE_FUSED). */
 KDA_API int kda_decode_engine(kda_handle h, int batch);
+
+/* Engine a kda_decode_step_tokens(batch, tokens) call runs (negative on bad arguments). */
+KDA_API int kda_decode_tokens_engine(kda_handle h, int batch, int tokens);
 
 /* Number of kernels one kda_decode_step(batch) launches. */
 KDA_API int kda_decode_launches_per_step(kda_handle h, int batch);

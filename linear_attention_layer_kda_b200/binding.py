@@ -34,7 +34,7 @@ EXPORTS = (
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
     "kda_decode_step_noalloc", "kda_decode_step_tokens", "kda_state_checkpoint", "kda_state_restore",
-    "kda_decode_set_launch_overlap",
+    "kda_decode_set_launch_overlap", "kda_decode_tokens_engine",
 )
 KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
 KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
@@ -96,6 +96,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_state_checkpoint": (I, [P, P, I, I, P]),
         "kda_state_restore": (I, [P, P, P, I, I]),
         "kda_decode_set_launch_overlap": (I, [P, I]),
+        "kda_decode_tokens_engine": (I, [P, I, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -156,6 +157,10 @@ def kda_decode_destroy(h: int) -> None:
 
 def kda_decode_engine(h: int, batch: int) -> int:
     return load().kda_decode_engine(h, batch)
+
+
+def kda_decode_tokens_engine(h: int, batch: int, tokens: int) -> int:
+    return load().kda_decode_tokens_engine(h, batch, tokens)
 
 
 def kda_decode_launches_per_step(h: int, batch: int) -> int:
@@ -296,6 +301,9 @@ class KdaDecoder:
 
     def engine(self, batch: int) -> int:
         return kda_decode_engine(self.h, batch)
+
+    def tokens_engine(self, batch: int, tokens: int) -> int:
+        return kda_decode_tokens_engine(self.h, batch, tokens)
 
     def launches_per_step(self, batch: int) -> int:
         return kda_decode_launches_per_step(self.h, batch)

@@ -99,6 +99,15 @@ int pick_engine(kda_handle h, int batch)
     return KDA_ENGINE_SIMPLE;
 }
 
+// Engine of a multi-token step: the fused kernel while it covers batch * tokens rows and
+// at most fused_max_tokens() tokens per sequence.
+int tokens_engine(kda_handle h, int batch, int tokens)
+{
+    if (tokens == 1) return pick_engine(h, batch);
+    if (tokens > kda::fused_max_tokens()) return KDA_ENGINE_SIMPLE;
+    return pick_engine(h, batch * tokens);
+}
+
 int check_weights(kda_handle h, const kda_weights *w)
 {
     if (!w) return fail(h, KDA_ERR_INVALID_ARG, "null weights");
@@ -159,7 +168,7 @@ int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state
     const kda::Dims d = dims_of(h->cfg, batch);
     cudaError_t e;
     if (pick_engine(h, batch) == KDA_ENGINE_FUSED)
-        e = kda::fused_step(d, *w, x, state, out, h->cfg.out_dtype, h->fused, h->s, h->status, h->stream);
+        e = kda::fused_step(d, 1, *w, x, state, out, h->cfg.out_dtype, h->fused, h->s, h->status, h->stream);
     else
         e = kda::simple_step(d, *w, x, state, out, h->cfg.out_dtype, h->s, h->stream);
     if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
@@ -406,6 +415,12 @@ int kda_decode_engine(kda_handle h, int batch)
     return pick_engine(h, batch);
 }
 
+int kda_decode_tokens_engine(kda_handle h, int batch, int tokens)
+{
+    if (!h || batch < 1 || tokens < 1 || (long long)batch * tokens > h->cfg.max_batch) return -KDA_ERR_INVALID_ARG;
+    return tokens_engine(h, batch, tokens);
+}
+
 int kda_decode_launches_per_step(kda_handle h, int batch)
 {
     if (!h || batch < 1 || batch > h->cfg.max_batch) return -KDA_ERR_INVALID_ARG;
@@ -471,8 +486,12 @@ int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, fl
         return fail(h, KDA_ERR_INVALID_ARG, "state_inout overlaps x or out");
     rc = take_device_status(h);
     if (rc) return rc;
-    const cudaError_t e = kda::simple_step_tokens(dims_of(c, batch), tokens, *w, x, state_inout, out, c.out_dtype,
-                                                  h->s, h->stream);
+    cudaError_t e;
+    if (tokens_engine(h, batch, tokens) == KDA_ENGINE_FUSED)
+        e = kda::fused_step(dims_of(c, batch * tokens), tokens, *w, x, state_inout, out, c.out_dtype, h->fused, h->s,
+                            h->status, h->stream);
+    else
+        e = kda::simple_step_tokens(dims_of(c, batch), tokens, *w, x, state_inout, out, c.out_dtype, h->s, h->stream);
     if (e != cudaSuccess) return cuda_fail(h, e, "kernel launch");
     return KDA_OK;
 }

@@ -59,6 +59,11 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 512;
+// Register shares per warpgroup (the block launches with 128 per thread): the single-lane
+// roles of warps 0-3 need few, the epilogue keeps 128, the state units get the rest.
+// 128 * (48 + 128 + 168 + 168) = 65536 = 512 * 128.
+constexpr int kRegsControl = 48, kRegsVector = 168;
+static_assert(kRegsControl + 128 + 2 * kRegsVector <= 4 * 128, "register shares exceed the launch budget");
 constexpr int kMaxBP = 64;
 constexpr int kMaxStages = 8;    // ring stages (weight tile + activation tile)
 constexpr int kMaxAcc = 4;       // TMEM accumulator buffers
@@ -106,15 +111,18 @@ constexpr int ST_CODE = 0, ST_WHERE = 1, ST_DRAIN = 2;
 
 constexpr int kOHand = 8;  // o-block hand-off barriers (state unit -> o publisher), reused mod 8
 
+constexpr int kMaxT = 8;  // tokens per sequence in one multi-token step
+
 struct __align__(16) VecSmem {
     uint64_t ohand[kOHand];        // unit k's o planes are stored (arrival of vector warp 0)
     int opub;                      // units whose o block the o publisher has released
     int pad_[3];
-    float q[256], k[256];          // per head of the unit: q, k^  (heads_per_unit * dk)
-    float a[2][256];               // alpha of the current and the next unit (by unit parity)
-    float v[128], u[128], o[128];  // per virtual column of the unit
-    float red_w[8][128], red_p[8][128];
-    float beta[2][2], kq[2], inv[2];  // beta: [unit parity][head of the unit]
+    float q[kMaxT][256], k[kMaxT][256];  // per token and head of the unit: q, k^ (heads_per_unit * dk)
+    float a[kMaxT][256];           // alpha per token (one token: slots of the current and next unit)
+    float v[kMaxT][128];           // per token and virtual column of the unit
+    float u[128], o[128];
+    float red_w[8][128], red_p[8][128];  // adjacent: also the t rows of token_gates
+    float beta[kMaxT][2], kq[kMaxT][2], inv[kMaxT][2];
     int unit, ok, fail;
 };
 
@@ -138,7 +146,8 @@ struct FusedParams {
     const uint32_t *cta_off;
     int *status;
     const uint2 *rbinfo;  // per row-group key: (first partial slot, segments)
-    int B, H, nh, dk, dv, r;
+    int B, H, nh, dk, dv, r;  // B: rows (sequences x tokens)
+    int T, Bs;                // tokens per sequence, sequences (B = Bs * T; row b * T + t)
     int nKBx, nKBo, nRGq, nRGv, nRGo;
     int off_oready, off_rb;
     uint32_t epoch, t_xq, t_gate, t_o;
@@ -442,7 +451,7 @@ __device__ void gate_rows(const FusedParams &P, VecSmem *vs, int vt)
 template <int DK>
 __device__ void unit_gates(const FusedParams &P, VecSmem *vs, int u, int slot, int vt, int t0, int nt)
 {
-    const int b = u % P.B, kb = u / P.B, hpu = 128 / P.dv, h0 = kb * hpu;
+    const int b = u % P.Bs, kb = u / P.Bs, hpu = 128 / P.dv, h0 = kb * hpu;
     const int me = vt - t0;
     if (me < 0 || me >= nt) return;
     if (me < hpu) vs->beta[slot][me] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + me)));
@@ -488,18 +497,18 @@ __device__ void first_gates(const FusedParams &P, VecSmem *vs, int u0, int u1, i
         const int j = vt / r4, c4 = vt % r4;
         if (us[j] >= 0)
             *reinterpret_cast<float4 *>(ts + j * P.r + 4 * c4) =
-                __ldcg(reinterpret_cast<const float4 *>(P.t + (size_t)(us[j] % P.B) * P.r) + c4);
+                __ldcg(reinterpret_cast<const float4 *>(P.t + (size_t)(us[j] % P.Bs) * P.r) + c4);
     } else if (vt >= 128 && vt < 128 + 2 * hpu) {
         const int j = (vt - 128) / hpu, hh = (vt - 128) % hpu;
         if (us[j] >= 0) {
-            const int b = us[j] % P.B, h = (us[j] / P.B) * hpu + hh;
+            const int b = us[j] % P.Bs, h = (us[j] / P.Bs) * hpu + hh;
             vs->beta[j][hh] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h)));
         }
     }
     for (int idx0 = 0; idx0 < 2 * rows; idx0 += 256) {
         const int idx = idx0 + vt, j = idx / rows, i = idx % rows;
         const bool has = idx < 2 * rows && us[j < 2 ? j : 0] >= 0;
-        const uint16_t *wr = P.wa_up + ((size_t)((has ? us[j] : 0) / P.B) * hpu * DK + i) * P.r;
+        const uint16_t *wr = P.wa_up + ((size_t)((has ? us[j] : 0) / P.Bs) * hpu * DK + i) * P.r;
         float z = 0.f;
         for (int j0 = 0; j0 < P.r; j0 += 64) {
             uint4 w4[8];
@@ -527,24 +536,87 @@ __device__ void first_gates(const FusedParams &P, VecSmem *vs, int u0, int u1, i
     named_bar(2, 256);
 }
 
-// One state unit: sequence b, o K-block kb (heads kb*128/dv ..), all dk rows.  Its gates are
-// in slot nu & 1; while a few threads wait for the unit's q/k/v, the others compute the gates
-// of this CTA's next unit (next_u >= 0) into the other slot.
-template <int BP, int DK>
+// Gates of every token of a multi-token unit (sequence bs, o K-block kb): alpha into a[t],
+// beta into beta[t].  Each thread loads one W_a_up row once and dots it with the T rows of t
+// (staged in shared memory).  t and W_b x must be final.
+template <int DK>
+__device__ void token_gates(const FusedParams &P, VecSmem *vs, int bs, int kb, int vt)
+{
+    const int T = P.T, hpu = 128 / P.dv, rows = hpu * DK, h0 = kb * hpu, r4 = P.r / 4;
+    float *ts = &vs->red_w[0][0];  // [T][r], T * r <= 2048 (red_w and red_p)
+    for (int idx = vt; idx < T * r4; idx += 256) {
+        const int t = idx / r4, c4 = idx % r4;
+        *reinterpret_cast<float4 *>(ts + t * P.r + 4 * c4) =
+            __ldcg(reinterpret_cast<const float4 *>(P.t + (size_t)(bs * T + t) * P.r) + c4);
+    }
+    for (int idx = vt; idx < T * hpu; idx += 256) {
+        const int t = idx / hpu, hh = idx % hpu;
+        vs->beta[t][hh] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)(bs * T + t) * P.nh + h0 + hh)));
+    }
+    for (int i0 = 0; i0 < rows; i0 += 256) {
+        const int i = i0 + vt;
+        const bool has = i < rows;
+        const uint16_t *wr = P.wa_up + ((size_t)h0 * DK + (has ? i : 0)) * P.r;
+        float z[kMaxT];
+#pragma unroll
+        for (int t = 0; t < kMaxT; ++t) z[t] = 0.f;
+        for (int j0 = 0; j0 < P.r; j0 += 64) {
+            uint4 w4[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                w4[q] = has && j0 + q * 8 < P.r ? __ldg(reinterpret_cast<const uint4 *>(wr + j0 + q * 8))
+                                                : make_uint4(0, 0, 0, 0);
+            if (i0 == 0 && j0 == 0) named_bar(2, 256);  // the t rows are in shared memory
+            if (!has) continue;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (j0 + q * 8 >= P.r) break;
+                const uint32_t wv[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
+                float wf[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    wf[2 * e] = bf16_bits_to_float(wv[e] & 0xFFFFu);
+                    wf[2 * e + 1] = bf16_bits_to_float(wv[e] >> 16);
+                }
+#pragma unroll
+                for (int t = 0; t < kMaxT; ++t) {
+                    if (t >= T) break;
+                    const float *tv = ts + t * P.r + j0 + q * 8;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) z[t] = fmaf(wf[e], tv[e], z[t]);
+                }
+            }
+        }
+        if (has)
+#pragma unroll
+            for (int t = 0; t < kMaxT; ++t)
+                if (t < T) vs->a[t][i] = 1.f / (1.f + expf(z[t]));
+    }
+    named_bar(2, 256);
+}
+
+// One state unit: sequence bs, o K-block kb (heads kb*128/dv ..), all dk rows, and its T
+// tokens applied in order (rows bs*T + t) with the state held in registers.  With one token
+// its gates are in slot nu & 1 and, while a few threads wait for the unit's q/k/v, the others
+// compute the gates of this CTA's next unit (next_u >= 0) into the other slot; with several
+// tokens every token's gates are computed here.
+template <int BP, int DK, bool MT>
 __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int u, int next_u, int vt, int nu)
 {
     constexpr ActGeo G = act_geo(BP);
-    const int b = u % P.B, kb = u / P.B, slot = nu & 1;
+    const int T = MT ? P.T : 1, bs = u % P.Bs, kb = u / P.Bs, slot = nu & 1;
     constexpr int RPW = DK / 8;  // rows per warp
     const int vw = vt >> 5, lane = vt & 31;
     const int dv = P.dv, hpu = 128 / dv, h0 = kb * hpu;
     const int vc = lane * 4, hh = vc / dv, cc = vc % dv, h = h0 + hh;
     const int Dk = P.nh * DK, Dv = P.nh * dv;
-    float *S = P.state + (((size_t)b * P.nh + h) * DK) * dv + cc;
+    float *S = P.state + (((size_t)bs * P.nh + h) * DK) * dv + cc;
 
     float4 s[RPW];
+    if (!MT) {
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) s[r] = ld_stream_f4(S + (size_t)(vw * RPW + r) * dv);
+        for (int r = 0; r < RPW; ++r) s[r] = ld_stream_f4(S + (size_t)(vw * RPW + r) * dv);
+    }
 
     if (vt == 0) vs->fail = 0;
     named_bar(2, 256);
@@ -558,30 +630,36 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
                                     : (vt < 2 * nq ? P.nRGq + glo + (vt - nq) : 2 * P.nRGq + vlo + (vt - 2 * nq));
             if (!wait_rb(P, key, c, 11)) vs->fail = 1;
         }
-        if (next_u >= 0 && nu >= 1) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
+        if (!MT && next_u >= 0 && nu >= 1) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
     }
     named_bar(2, 256);
-    if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
+    if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
     if (vs->fail) return false;
+    if (MT) {
+        token_gates<DK>(P, vs, bs, kb, vt);
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) s[r] = ld_stream_f4(S + (size_t)(vw * RPW + r) * dv);
+    }
+    const int nqk = hpu * DK, per = 2 * nqk + 128;
     {
-        // items: q and k rows of the unit's heads, then its 128 v columns; a thread's items
-        // are loaded together (one memory round trip), then summed in slot order
-        const int nqk = hpu * DK, nitems = 2 * nqk + 128;
+        // items (token t, i): q and k rows of the unit's heads, then its 128 v columns; a
+        // thread's items are loaded together (one memory round trip), then summed in slot order
+        const int nitems = T * per;
         for (int it0 = 0; it0 < nitems; it0 += 512) {
             int key[2], off[2];
             bool has[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int it = it0 + vt + 256 * j;
+                const int it = it0 + vt + 256 * j, t = it / per, i = it % per, row = bs * T + t;
                 has[j] = it < nitems;
-                if (it < 2 * nqk) {
-                    const int row = h0 * DK + it % nqk;
-                    key[j] = (it / nqk) * P.nRGq + row / G.nx;
-                    off[j] = b * G.nx + row % G.nx;
+                if (i < 2 * nqk) {
+                    const int qrow = h0 * DK + i % nqk;
+                    key[j] = (i / nqk) * P.nRGq + qrow / G.nx;
+                    off[j] = row * G.nx + qrow % G.nx;
                 } else {
-                    const int col = kb * 128 + (it - 2 * nqk);
+                    const int col = kb * 128 + (i - 2 * nqk);
                     key[j] = 2 * P.nRGq + col / G.nx;
-                    off[j] = b * G.nx + col % G.nx;
+                    off[j] = row * G.nx + col % G.nx;
                 }
             }
             float val[2];
@@ -589,104 +667,114 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
             if (vt == 0 && nu < 2 && it0 == 0) KDA_TR(P, TR_UNIT_SUMS + nu);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int it = it0 + vt + 256 * j;
+                const int it = it0 + vt + 256 * j, t = it / per, i = it % per, row = bs * T + t;
                 if (!has[j]) continue;
-                if (it < 2 * nqk) {
-                    const int i = it % nqk, isk = it / nqk, row = h0 * DK + i;
-                    (isk ? vs->k : vs->q)[i] = val[j];
-                    (isk ? P.k : P.q)[(size_t)b * Dk + row] = val[j];  // kept for kda_decode_debug_copy
+                if (i < 2 * nqk) {
+                    const int ii = i % nqk, isk = i / nqk, qrow = h0 * DK + ii;
+                    (isk ? vs->k[t] : vs->q[t])[ii] = val[j];
+                    (isk ? P.k : P.q)[(size_t)row * Dk + qrow] = val[j];  // kept for kda_decode_debug_copy
                 } else {
-                    const int i = it - 2 * nqk;
-                    vs->v[i] = val[j];
-                    P.v[(size_t)b * Dv + (size_t)kb * 128 + i] = val[j];
+                    const int ii = i - 2 * nqk;
+                    vs->v[t][ii] = val[j];
+                    P.v[(size_t)row * Dv + (size_t)kb * 128 + ii] = val[j];
                 }
             }
         }
     }
     named_bar(2, 256);
     if (vt == 0 && nu == 0) KDA_TR(P, TR_UNIT_ITEMS);
-    // ||k|| and k.q per head (one warp per head)
-    if (vw < hpu) {
+    // ||k|| and k.q per token and head (one warp per pair)
+    for (int pr = vw; pr < T * hpu; pr += 8) {
+        const int t = pr / hpu, hd = pr % hpu;
         float ss = 0.f, kq = 0.f;
         for (int i = lane; i < DK; i += 32) {
-            const float kv = vs->k[vw * DK + i];
+            const float kv = vs->k[t][hd * DK + i];
             ss = fmaf(kv, kv, ss);
-            kq = fmaf(kv, vs->q[vw * DK + i], kq);
+            kq = fmaf(kv, vs->q[t][hd * DK + i], kq);
         }
         ss = warp_sum(ss);
         kq = warp_sum(kq);
         if (lane == 0) {
             const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
-            vs->inv[vw] = inv;
-            vs->kq[vw] = kq * inv;
+            vs->inv[t][hd] = inv;
+            vs->kq[t][hd] = kq * inv;
         }
     }
     named_bar(2, 256);
-    for (int i = vt; i < hpu * DK; i += 256) vs->k[i] *= vs->inv[i / DK];
+    for (int i = vt; i < T * nqk; i += 256) vs->k[i / nqk][i % nqk] *= vs->inv[i / nqk][(i % nqk) / DK];
     named_bar(2, 256);
 
-    // S~ = diag(alpha) S; partial w = S~^T k^, p = S~^T q over this warp's rows
-    float4 pw = make_float4(0.f, 0.f, 0.f, 0.f), pp = pw;
+    for (int t = 0; t < T; ++t) {
+        const float *al = vs->a[MT ? t : slot];
+        const float *kt = vs->k[t], *qt = vs->q[t];
+        // S~ = diag(alpha) S; partial w = S~^T k^, p = S~^T q over this warp's rows
+        float4 pw = make_float4(0.f, 0.f, 0.f, 0.f), pp = pw;
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-        const int i = hh * DK + vw * RPW + r;
-        const float a = vs->a[slot][i], kk = vs->k[i], qq = vs->q[i];
-        s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
-        pw.x = fmaf(kk, s[r].x, pw.x); pw.y = fmaf(kk, s[r].y, pw.y);
-        pw.z = fmaf(kk, s[r].z, pw.z); pw.w = fmaf(kk, s[r].w, pw.w);
-        pp.x = fmaf(qq, s[r].x, pp.x); pp.y = fmaf(qq, s[r].y, pp.y);
-        pp.z = fmaf(qq, s[r].z, pp.z); pp.w = fmaf(qq, s[r].w, pp.w);
-    }
-    *reinterpret_cast<float4 *>(&vs->red_w[vw][vc]) = pw;
-    *reinterpret_cast<float4 *>(&vs->red_p[vw][vc]) = pp;
-    named_bar(2, 256);
-    if (vt < 128) {
-        float w = 0.f, p = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            w += vs->red_w[j][vt];
-            p += vs->red_p[j][vt];
+        for (int r = 0; r < RPW; ++r) {
+            const int i = hh * DK + vw * RPW + r;
+            const float a = al[i], kk = kt[i], qq = qt[i];
+            s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
+            pw.x = fmaf(kk, s[r].x, pw.x); pw.y = fmaf(kk, s[r].y, pw.y);
+            pw.z = fmaf(kk, s[r].z, pw.z); pw.w = fmaf(kk, s[r].w, pw.w);
+            pp.x = fmaf(qq, s[r].x, pp.x); pp.y = fmaf(qq, s[r].y, pp.y);
+            pp.z = fmaf(qq, s[r].z, pp.z); pp.w = fmaf(qq, s[r].w, pp.w);
         }
-        const int hx = vt / dv;
-        const float uu = vs->beta[slot][hx] * (vs->v[vt] - w);
-        vs->u[vt] = uu;
-        vs->o[vt] = fmaf(uu, vs->kq[hx], p);
-    }
-    named_bar(2, 256);
-    if (vt == 0 && nu == 0) KDA_TR(P, TR_UNIT_O);
-    // o -> four E4M3 planes with one power-of-two scale for the K-block; release it
-    if (vw == 0) {
-        const float4 o4 = *reinterpret_cast<const float4 *>(&vs->o[vc]);
-        const float amax = warp_max(fmaxf(fmaxf(fabsf(o4.x), fabsf(o4.y)), fmaxf(fabsf(o4.z), fabsf(o4.w))));
-        const float sc = pow2_scale(amax), inv = 1.f / sc;
-        uint32_t wq[4];
-        split_planes<4>(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv, wq);
+        *reinterpret_cast<float4 *>(&vs->red_w[vw][vc]) = pw;
+        *reinterpret_cast<float4 *>(&vs->red_p[vw][vc]) = pp;
+        named_bar(2, 256);
+        if (vt < 128) {
+            float w = 0.f, p = 0.f;
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
-            *reinterpret_cast<uint32_t *>(P.oq + (size_t)o_row(p, b) * Dv + (size_t)kb * 128 + vc) = wq[p];
-        if (lane == 0)
-            *reinterpret_cast<float *>(P.oq + (size_t)(G.rso + b / 32) * Dv + (size_t)kb * 128 + (b % 32) * 4) = sc;
-        fence_proxy_async_global();
+            for (int j = 0; j < 8; ++j) {
+                w += vs->red_w[j][vt];
+                p += vs->red_p[j][vt];
+            }
+            const int hx = vt / dv;
+            const float uu = vs->beta[MT ? t : slot][hx] * (vs->v[t][vt] - w);
+            vs->u[vt] = uu;
+            vs->o[vt] = fmaf(uu, vs->kq[t][hx], p);
+        }
+        named_bar(2, 256);
+        if (vt == 0 && nu == 0 && t == 0) KDA_TR(P, TR_UNIT_O);
+        // o of row bs*T + t -> four E4M3 planes with one power-of-two scale for the K-block
+        if (vw == 0) {
+            const int row = bs * T + t;
+            const float4 o4 = *reinterpret_cast<const float4 *>(&vs->o[vc]);
+            const float amax = warp_max(fmaxf(fmaxf(fabsf(o4.x), fabsf(o4.y)), fmaxf(fabsf(o4.z), fabsf(o4.w))));
+            const float sc = pow2_scale(amax), inv = 1.f / sc;
+            uint32_t wq[4];
+            split_planes<4>(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv, wq);
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+                *reinterpret_cast<uint32_t *>(P.oq + (size_t)o_row(p, row) * Dv + (size_t)kb * 128 + vc) = wq[p];
+            if (lane == 0)
+                *reinterpret_cast<float *>(P.oq + (size_t)(G.rso + row / 32) * Dv + (size_t)kb * 128 + (row % 32) * 4) = sc;
+            fence_proxy_async_global();
+        }
+        // S' = S~ + k^ u^T (kept in registers for the next token)
+        const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+            const float kk = kt[hh * DK + vw * RPW + r];
+            s[r].x = fmaf(kk, u4.x, s[r].x); s[r].y = fmaf(kk, u4.y, s[r].y);
+            s[r].z = fmaf(kk, u4.z, s[r].z); s[r].w = fmaf(kk, u4.w, s[r].w);
+        }
+        if (t + 1 < T) named_bar(2, 256);  // u, o and the reductions are reused by the next token
+    }
+    if (vw == 0) {
         __syncwarp();
         if (lane == 0) {
-            // hand the release to the o publisher (its fence then never holds up the unit); at
-            // most kOHand units may wait for it
+            // hand the release of the o block (every token's planes) to the o publisher (its
+            // fence then never holds up the unit); at most kOHand units may wait for it
             const uint64_t t0 = globaltimer_ns();
             while (nu - *(volatile int *)&vs->opub >= kOHand && globaltimer_ns() - t0 < P.timeout_ns) __nanosleep(64);
             mbar_arrive(&vs->ohand[nu % kOHand]);
             if (nu < 2) KDA_TR(P, TR_UNIT_HAND + nu);
         }
     }
-    // S' = S~ + k^ u^T, written back in place (after the hand-off: nothing reads it this step)
-    const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
+    // the updated state, written back in place (after the hand-off: nothing reads it this step)
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-        const float kk = vs->k[hh * DK + vw * RPW + r];
-        float4 o;
-        o.x = fmaf(kk, u4.x, s[r].x); o.y = fmaf(kk, u4.y, s[r].y);
-        o.z = fmaf(kk, u4.z, s[r].z); o.w = fmaf(kk, u4.w, s[r].w);
-        st_stream_f4(S + (size_t)(vw * RPW + r) * dv, o);
-    }
+    for (int r = 0; r < RPW; ++r) st_stream_f4(S + (size_t)(vw * RPW + r) * dv, s[r]);
     named_bar(2, 256);
     return true;
 }
@@ -695,10 +783,10 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 // warp 0 has stored their planes.
 __device__ void o_publisher(const FusedParams &P, VecSmem *vs, const Ctl &c)
 {
-    const int units = P.B * P.nKBo;
+    const int units = P.Bs * P.nKBo;
     for (int k = 0, u = blockIdx.x; u < units; ++k, u += gridDim.x) {
         if (!wait_bar(&vs->ohand[k % kOHand], (uint32_t)(k / kOHand) & 1u, c, 14)) return;
-        if (!*c.sh_abort) red_release_add(P.ctr + P.off_oready + u / P.B, 1u);
+        if (!*c.sh_abort) red_release_add(P.ctr + P.off_oready + u / P.Bs, 1u);
         *(volatile int *)&vs->opub = k + 1;
     }
 }
@@ -706,7 +794,7 @@ __device__ void o_publisher(const FusedParams &P, VecSmem *vs, const Ctl &c)
 // State of unit u (sequence u % B, the heads of o K-block u / B) -> L2, in 32 KB bulk prefetches.
 __device__ void prefetch_unit_state(const FusedParams &P, int u)
 {
-    const int b = u % P.B, kb = u / P.B, hpu = 128 / P.dv;
+    const int b = u % P.Bs, kb = u / P.Bs, hpu = 128 / P.dv;
     const size_t bytes = (size_t)hpu * P.dk * P.dv * 4;
     const char *p = reinterpret_cast<const char *>(P.state + (((size_t)b * P.nh + (size_t)kb * hpu) * P.dk) * P.dv);
     const uint64_t pol = policy_evict_last();
@@ -714,26 +802,26 @@ __device__ void prefetch_unit_state(const FusedParams &P, int u)
         bulk_prefetch_l2_hint(p + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
 }
 
-template <int BP, int DK>
+template <int BP, int DK, bool MT>
 __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
 {
     constexpr ActGeo G = act_geo(BP);
     const int vt = threadIdx.x - 256, vw = vt >> 5, lane = vt & 31;
     quantize_x<BP>(P, blockIdx.x * 8 + vw, gridDim.x * 8, lane);
     if (vt == 0) KDA_TR(P, TR_XQ_DONE);
-    if (vt == 0 && (int)blockIdx.x < P.B * P.nKBo) prefetch_unit_state(P, blockIdx.x);
+    if (vt == 0 && (int)blockIdx.x < P.Bs * P.nKBo) prefetch_unit_state(P, blockIdx.x);
     gate_rows<BP>(P, vs, vt);
     if (vt == 0) KDA_TR(P, TR_GATES_DONE);
     // State units (sequence u % B, o K-block u / B) in head order, CTA c taking c, c + grid,
     // ...: the same units every step, so the next unit's gates are computed while the
     // current one waits for its q/k/v.
-    const int units = P.B * P.nKBo;
+    const int units = P.Bs * P.nKBo;
     if ((int)blockIdx.x < units) {
         if (vt == 0) vs->ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);  // t and W_b x final
         named_bar(2, 256);
         if (!vs->ok) return;
         const int u1 = (int)(blockIdx.x + gridDim.x);
-        first_gates<DK>(P, vs, blockIdx.x, u1 < units ? u1 : -1, vt);
+        if (!MT) first_gates<DK>(P, vs, blockIdx.x, u1 < units ? u1 : -1, vt);  // else per unit
     }
     for (int nu = 0, u = blockIdx.x; u < units; ++nu, u += gridDim.x) {
         if (vt == 0) vs->unit = should_stop(c) ? 1 : 0;
@@ -742,7 +830,7 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
         if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu);
         const int next = u + (int)gridDim.x < units ? u + (int)gridDim.x : -1;
         if (vt == 0 && next >= 0) prefetch_unit_state(P, next);  // its state streams in meanwhile
-        if (!state_unit<BP, DK>(P, vs, c, u, next, vt, nu)) return;
+        if (!state_unit<BP, DK, MT>(P, vs, c, u, next, vt, nu)) return;
         if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
     }
     // out = sum of the W_o partials (both plane pairs): items of 32 output rows
@@ -1109,7 +1197,9 @@ __device__ void publisher(const FusedParams &P, const Ring &R, const TileEntry *
     }
 }
 
-template <int BP, int DK>
+// MT: several tokens per sequence (multi-token steps; a separate instantiation keeps the
+// single-token state unit's registers to itself)
+template <int BP, int DK, bool MT>
 __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ FusedParams P)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -1187,23 +1277,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == 3 && lane == 0) prefetch_l2_slice(P.x, (size_t)P.B * P.H * 2);
 
-    if (warp == 0) {
-        if (lane == 0) producer<BP>(P, R, my, n, c, pre);
+    if (warp < 4) {  // single-lane roles: few registers
+        regs_dec<kRegsControl>();
+        if (warp == 0) {
+            if (lane == 0) producer<BP>(P, R, my, n, c, pre);
+        } else if (warp == 1) {
+            if (lane == 0) o_publisher(P, vs, c);
+        } else if (warp == 2) {
+            if (lane == 0) mma_issuer<BP>(P, R, my, n, tmem, c);
+        } else {
+            if (lane == 0) publisher(P, R, my, n, c);
+        }
         __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0) o_publisher(P, vs, c);
-        __syncwarp();
-    } else if (warp == 2) {
-        if (lane == 0) mma_issuer<BP>(P, R, my, n, tmem, c);
-        __syncwarp();
-    } else if (warp == 3) {
-        if (lane == 0) publisher(P, R, my, n, c);
-        __syncwarp();
-    } else if (warp >= 4 && warp < 4 + kEpiWarps) {
+    } else if (warp < 4 + kEpiWarps) {
         epilogue_role<BP>(P, R, my, n, tmem, c);
         if (threadIdx.x == 128) KDA_TR(P, TR_EPI_DONE);
-    } else if (warp >= 8) {
-        vector_role<BP, DK>(P, vs, c);
+    } else {  // state units: the registers the others gave up
+        regs_inc<kRegsVector>();
+        vector_role<BP, DK, MT>(P, vs, c);
     }
     tc_fence_before();
     __syncthreads();
@@ -1286,23 +1377,25 @@ int row_group_keys(const Dims &d, const SchedGeo &g)
 
 size_t ctr_words(const Dims &d, int max_keys) { return C_FIXED + (size_t)d.Dv() / 128 + max_keys + 16; }
 
-template <int BP, int DK>
-void *kernel_ptr() { return reinterpret_cast<void *>(&k_fused<BP, DK>); }
+template <int BP, int DK, bool MT>
+void *kernel_ptr() { return reinterpret_cast<void *>(&k_fused<BP, DK, MT>); }
 
-void *pick_kernel(int BP, int DK)
+template <bool MT>
+void *pick_kernel_t(int BP, int DK)
 {
     switch (BP * 1000 + DK) {
-    case 8064: return kernel_ptr<8, 64>();
-    case 8128: return kernel_ptr<8, 128>();
-    case 16064: return kernel_ptr<16, 64>();
-    case 16128: return kernel_ptr<16, 128>();
-    case 32064: return kernel_ptr<32, 64>();
-    case 32128: return kernel_ptr<32, 128>();
-    case 64064: return kernel_ptr<64, 64>();
-    case 64128: return kernel_ptr<64, 128>();
+    case 8064: return kernel_ptr<8, 64, MT>();
+    case 8128: return kernel_ptr<8, 128, MT>();
+    case 16064: return kernel_ptr<16, 64, MT>();
+    case 16128: return kernel_ptr<16, 128, MT>();
+    case 32064: return kernel_ptr<32, 64, MT>();
+    case 32128: return kernel_ptr<32, 128, MT>();
+    case 64064: return kernel_ptr<64, 64, MT>();
+    case 64128: return kernel_ptr<64, 128, MT>();
     default: return nullptr;
     }
 }
+void *pick_kernel(int BP, int DK, bool multi) { return multi ? pick_kernel_t<true>(BP, DK) : pick_kernel_t<false>(BP, DK); }
 
 size_t fixed_smem_bytes(int max_tiles)
 {
@@ -1451,12 +1544,15 @@ void fused_destroy(FusedState *fs)
 
 int fused_launches() { return 1; }
 
-cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float *state, void *out, int out_dtype,
-                       FusedState &fs, const Scratch &s, int *status, cudaStream_t stream)
+int fused_max_tokens() { return kMaxT; }
+
+cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const void *x, float *state, void *out,
+                       int out_dtype, FusedState &fs, const Scratch &s, int *status, cudaStream_t stream)
 {
     if (!fs.uploaded) return cudaErrorNotReady;
+    if (tokens < 1 || tokens > kMaxT || d.B % tokens) return cudaErrorNotSupported;
     const int BP = bp_for(d.B), cls = class_of(BP);
-    void *kern = pick_kernel(BP, d.dk);
+    void *kern = pick_kernel(BP, d.dk, tokens > 1);
     if (!kern || cls >= fs.nclass) return cudaErrorNotSupported;
     const ActGeo g = act_geo(BP);
     const SchedGeo sg = fused_sched_geo(d, BP);
@@ -1466,6 +1562,7 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
         if (e != cudaSuccess) return e;
         fs.epoch = 0;
         fs.cum_b = 0;
+        fs.cum_s = 0;
         fs.needs_reset = false;
     }
     static thread_local FusedParams P;
@@ -1537,6 +1634,8 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.cta_off = fs.cta_off[cls];
     P.status = status;
     P.B = d.B;
+    P.T = tokens;
+    P.Bs = d.B / tokens;
     P.H = d.H;
     P.nh = d.nh;
     P.dk = d.dk;
@@ -1555,7 +1654,7 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     P.t_xq = (fs.cum_b + (uint32_t)d.B) * (uint32_t)P.nKBx;
     P.early_tiles = fs.early_tiles;
     P.t_gate = epoch * (uint32_t)(d.nh + d.r);
-    P.t_o = fs.cum_b + (uint32_t)d.B;
+    P.t_o = fs.cum_s + (uint32_t)P.Bs;
     P.timeout_ns = fs.timeout_ns;
     P.out_bf16 = out_dtype == KDA_OUT_BF16;
     P.skip_gate_release = fs.debug_skip_gate_release;
@@ -1610,6 +1709,7 @@ cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float
     fs.last_class = cls;
     fs.epoch = epoch;
     fs.cum_b += (uint32_t)d.B;
+    fs.cum_s += (uint32_t)P.Bs;
     return cudaSuccess;
 }
 

@@ -98,7 +98,8 @@ struct FusedState {
     std::vector<uint32_t> h_rbinfo[4];
     int last_class = -1;            // class of the previous step (counters are per class)
     uint32_t epoch = 0;  // steps issued since the last reset
-    uint32_t cum_b = 0;  // sum of batch sizes of those steps
+    uint32_t cum_b = 0;  // sum of rows (sequences x tokens) of those steps
+    uint32_t cum_s = 0;  // sum of sequences of those steps
     bool needs_reset = false;
     bool uploaded = false;
     uint64_t timeout_ns = 2000000000ull;
@@ -125,8 +126,10 @@ void fused_bind_scratch(const Dims &dmax, int num_sms, void *base, size_t bytes,
 cudaError_t fused_init(const Dims &dmax, FusedState *fs);
 void fused_destroy(FusedState *fs);
 int fused_launches();
-cudaError_t fused_step(const Dims &d, const kda_weights &w, const void *x, float *state, void *out, int out_dtype,
-                       FusedState &fs, const Scratch &s, int *status, cudaStream_t stream);
+int fused_max_tokens();
+// d.B rows = sequences x tokens (row b * tokens + t); tokens <= fused_max_tokens().
+cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const void *x, float *state, void *out,
+                       int out_dtype, FusedState &fs, const Scratch &s, int *status, cudaStream_t stream);
 
 // Schedule shape of a step whose padded batch is BP (host only).
 SchedGeo fused_sched_geo(const Dims &dmax, int BP);

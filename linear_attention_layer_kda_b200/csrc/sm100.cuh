@@ -190,6 +190,14 @@ __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t *p, uint32_t v)
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
+// Per-warpgroup register budget (all four warps of a warpgroup execute the same one).  The
+// shares of the block's warpgroups must add up to no more than the registers it was launched
+// with, or an increase waits forever.
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
 __device__ __forceinline__ void named_bar(int id, int nthreads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
