@@ -318,7 +318,7 @@ def run_ours(args, shape, rank, world, local_rank):
     props = torch.cuda.get_device_properties(dev)
     l2 = max(L2_ASSUMED, int(getattr(props, "L2_cache_size", L2_ASSUMED)))
 
-    TK = args.tokens
+    TK = args.tokens if args.prefill <= 0 else args.prefill
     if TK > 1:
         shape = shape.replace(steps=max(shape.steps, TK))
     inp = rank_inputs(shape, rank, world)
@@ -334,14 +334,20 @@ def run_ours(args, shape, rank, world, local_rank):
     else:
         xs = [tensors.bf16_tensor(inp.x[t], dev) for t in range(T)]
     outs = [torch.empty(B * TK, shape.hidden, device=dev, dtype=torch.float32) for _ in range(R)]
-    dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, B * TK,
-                             engine=args.engine)
-    engine = dec.engine(B) if TK == 1 else dec.tokens_engine(B, TK)
-    launches = dec.launches_per_step(B) if TK == 1 else (1 if engine == 2 else dec.launches_per_step(B))
+    prefill = args.prefill > 0
+    dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank,
+                             B if prefill else B * TK, engine=args.engine)
+    if prefill:
+        engine, launches = "prefill", 5  # three projection launches, the chunk kernel, W_o
+    else:
+        engine = dec.engine(B) if TK == 1 else dec.tokens_engine(B, TK)
+        launches = dec.launches_per_step(B) if TK == 1 else (1 if engine == 2 else dec.launches_per_step(B))
 
     def one(i):
         j = i % R
-        if TK == 1:
+        if prefill:
+            dec.prefill(xs[0], ws[j], states[j], outs[j], B, TK, args.chunk)
+        elif TK == 1:
             dec.step(xs[i % T], ws[j], states[j], outs[j])
         else:
             dec.step_tokens(xs[0], ws[j], states[j], outs[j], B, TK)
@@ -462,6 +468,7 @@ def run_ours(args, shape, rank, world, local_rank):
                             "the events also stop consecutive steps from overlapping"},
         "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
         "engine": {1: "simple", 2: "fused"}.get(engine, str(engine)),
+        **({"prefill": {"tokens": TK, "chunk": args.chunk or 32}} if prefill else {}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
                      "peak_source": f"{peak_src} copy bandwidth",
@@ -473,7 +480,7 @@ def run_ours(args, shape, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "cpu_baseline": cpu,
-        "ideal_flops_per_step": ideal_flops(shape, B),
+        "ideal_flops_per_step": ideal_flops(shape, B * TK),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -522,6 +529,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the host-buffer end-to-end loop")
     ap.add_argument("--tokens", type=int, default=1,
                     help="tokens per sequence in one step (multi-token verify through kda_decode_step_tokens)")
+    ap.add_argument("--prefill", type=int, default=0, help="time kda_prefill of this many tokens per sequence")
+    ap.add_argument("--chunk", type=int, default=0, help="prefill chunk (16, 32, 64; 0: the library default)")
     ap.add_argument("--launch-limit", type=int, default=900, help="seconds before a self-launched job is killed")
     ap.add_argument("--print-rank", action="store_true", help=argparse.SUPPRESS)  # launcher self-check
     return ap.parse_args(argv)

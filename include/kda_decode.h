@@ -172,6 +172,26 @@ KDA_API int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weight
                                    int batch, int tokens);
 
 /*
+ * Prefill: `tokens` consecutive tokens of each of `batch` sequences (a prompt), through the
+ * chunked form of the recurrence -- the parallel-in-time prefill form that the Kiln post names
+ * among its KDA kernels ("What moved the number...", "The token mixers' collectives...").
+ *   x            bf16 [batch * tokens, H]; row b * tokens + t is token t of sequence b
+ *   state_inout  fp32 [batch, nh, dk, dv]; advanced by all `tokens` tokens
+ *   out          [batch * tokens, H] (cfg.out_dtype); row b * tokens + t is the output of
+ *                token t, read out after token t's update
+ *   chunk        tokens per chunk: 16, 32 or 64 (0: 32)
+ * Each head's state goes through the tokens `chunk` at a time: inside a chunk the tokens'
+ * updates are one unit lower-triangular solve and dense products (decays taken in log space,
+ * log alpha clamped at -30).  The projections run the five-kernel engine's GEMV kernels over
+ * all rows.  batch and tokens are not limited by max_batch: the handle keeps a workspace of
+ * the activations of batch * tokens rows, allocated (cudaMalloc; waiting for the device when
+ * it grows) on the first call that needs it and freed by kda_decode_destroy.  Same errors
+ * and stream ordering as kda_decode_step; KDA_ERR_OUT_OF_MEMORY if the workspace cannot grow.
+ */
+KDA_API int kda_prefill(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out, int batch,
+                        int tokens, int chunk);
+
+/*
  * Recurrent-state checkpoint and restore (the Kiln post's prefix cache keeps checkpoints of
  * linear-attention state in a host tier: "What is Kiln?"; its "What could only a device
  * show?" is the lesson that such a copy must be ordered behind the queued work).  Both are

@@ -34,7 +34,7 @@ EXPORTS = (
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
     "kda_decode_step_noalloc", "kda_decode_step_tokens", "kda_state_checkpoint", "kda_state_restore",
-    "kda_decode_set_launch_overlap", "kda_decode_tokens_engine",
+    "kda_decode_set_launch_overlap", "kda_decode_tokens_engine", "kda_prefill",
 )
 KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
 KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
@@ -97,6 +97,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_state_restore": (I, [P, P, P, I, I]),
         "kda_decode_set_launch_overlap": (I, [P, I]),
         "kda_decode_tokens_engine": (I, [P, I, I]),
+        "kda_prefill": (I, [P, P, ctypes.POINTER(kda_weights), P, P, I, I, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -129,6 +130,10 @@ def kda_decode_step(h: int, x: int, w: kda_weights, state: int, out: int, batch:
 
 def kda_decode_step_tokens(h: int, x: int, w: kda_weights, state: int, out: int, batch: int, tokens: int) -> None:
     _check(load().kda_decode_step_tokens(h, x, ctypes.byref(w), state, out, batch, tokens), "kda_decode_step_tokens", h)
+
+
+def kda_prefill(h: int, x: int, w: kda_weights, state: int, out: int, batch: int, tokens: int, chunk: int) -> None:
+    _check(load().kda_prefill(h, x, ctypes.byref(w), state, out, batch, tokens, chunk), "kda_prefill", h)
 
 
 def kda_state_checkpoint(h: int, state: int, seq0: int, nseq: int, host_dst: int) -> None:
@@ -258,6 +263,18 @@ class KdaDecoder:
             raise ValueError(f"x and out need {rows} rows and state {batch} sequences")
         self._bind_stream()
         kda_decode_step_tokens(self.h, x.data_ptr(), weights, state.data_ptr(), out.data_ptr(), batch, tokens)
+
+    def prefill(self, x, weights: kda_weights, state, out, batch: int, tokens: int, chunk: int = 0) -> None:
+        """`tokens` tokens of each of `batch` sequences through the chunked recurrence; x and out
+        are [batch * tokens, H]."""
+        for n, a in (("x", x), ("state", state), ("out", out)):
+            if not a.is_cuda or not a.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous CUDA tensor")
+        rows = batch * tokens
+        if x.shape[0] < rows or out.shape[0] < rows or state.shape[0] < batch:
+            raise ValueError(f"x and out need {rows} rows and state {batch} sequences")
+        self._bind_stream()
+        kda_prefill(self.h, x.data_ptr(), weights, state.data_ptr(), out.data_ptr(), batch, tokens, chunk)
 
     def _state_range(self, state, host, seq0: int, nseq: Optional[int]) -> int:
         n = state.shape[0] - seq0 if nseq is None else nseq

@@ -24,6 +24,8 @@ struct kda_handle_s {
     void *x_stage = nullptr;    // device staging of x for kda_decode_step_host
     void *out_stage = nullptr;  // device staging of out for kda_decode_step_host
     kda::FusedState fused;
+    void *pf_ws = nullptr;   // prefill workspace (activations of every row), grown on demand
+    size_t pf_bytes = 0;
     bool fatal = false;  // a kernel gave up draining its copies after an abort: never step again
     std::string last_error;
 };
@@ -496,6 +498,62 @@ int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, fl
     return KDA_OK;
 }
 
+int kda_prefill(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out, int batch,
+                int tokens, int chunk)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    if (int rc0 = check_usable(h)) return rc0;
+    const kda_config &c = h->cfg;
+    if (chunk == 0) chunk = 32;
+    if (batch < 1 || tokens < 1) return fail(h, KDA_ERR_INVALID_ARG, "batch and tokens must be >= 1");
+    if (!kda::chunk_supported(c.head_dk, c.head_dv, chunk))
+        return fail(h, KDA_ERR_INVALID_ARG, "chunk must be 16, 32 or 64");
+    if (!x || !state_inout || !out) return fail(h, KDA_ERR_INVALID_ARG, "null x, state or out");
+    if (!aligned16(x) || !aligned16(state_inout) || !aligned16(out))
+        return fail(h, KDA_ERR_INVALID_ARG, "x, state and out must be 16-byte aligned");
+    int rc = check_weights(h, w);
+    if (rc) return rc;
+    const long long rows_ll = (long long)batch * tokens;
+    const size_t Dk = (size_t)c.num_heads * c.head_dk, Dv = (size_t)c.num_heads * c.head_dv;
+    if (rows_ll > (1LL << 31) / (long long)(Dk > (size_t)c.hidden ? Dk : (size_t)c.hidden))
+        return fail(h, KDA_ERR_INVALID_ARG, "batch * tokens too large");
+    const size_t rows = (size_t)rows_ll;
+    const size_t nx = rows * c.hidden * 2, no = rows * c.hidden * (c.out_dtype == KDA_OUT_BF16 ? 2 : 4);
+    const size_t ns = (size_t)batch * c.num_heads * c.head_dk * c.head_dv * 4;
+    if (overlaps(state_inout, ns, x, nx) || overlaps(state_inout, ns, out, no))
+        return fail(h, KDA_ERR_INVALID_ARG, "state_inout overlaps x or out");
+    rc = take_device_status(h);
+    if (rc) return rc;
+    // workspace: the fp32 activations of every row
+    const size_t sizes[7] = {rows * Dk * 4, rows * Dk * 4, rows * Dk * 4, rows * Dv * 4, rows * Dv * 4,
+                             rows * (size_t)c.num_heads * 4, rows * (size_t)c.alpha_rank * 4};
+    size_t need = 0;
+    for (size_t sz : sizes) need += align_up(sz, 256);
+    if (need > h->pf_bytes) {
+        if (h->pf_ws && cudaFree(h->pf_ws) != cudaSuccess) (void)cudaGetLastError();  // waits for its users
+        h->pf_ws = nullptr;
+        h->pf_bytes = 0;
+        if (cudaMalloc(&h->pf_ws, need) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return fail(h, KDA_ERR_OUT_OF_MEMORY, "prefill workspace allocation failed");
+        }
+        h->pf_bytes = need;
+    }
+    kda::Scratch s;
+    float **dst[7] = {&s.q, &s.k, &s.z, &s.v, &s.o, &s.bpre, &s.t};
+    char *p = static_cast<char *>(h->pf_ws);
+    for (int i = 0; i < 7; ++i) {
+        *dst[i] = reinterpret_cast<float *>(p);
+        p += align_up(sizes[i], 256);
+    }
+    const kda::Dims d = dims_of(c, (int)rows);
+    cudaError_t e = kda::simple_projections(d, *w, x, s, h->stream);
+    if (e == cudaSuccess) e = kda::chunk_state(d, batch, tokens, chunk, s, state_inout, h->stream);
+    if (e == cudaSuccess) e = kda::simple_out_projection(d, *w, s.o, out, c.out_dtype, h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "prefill launch");
+    return KDA_OK;
+}
+
 static int state_copy(kda_handle h, void *dst, const void *src, int seq0, int nseq, bool to_host)
 {
     if (!h) return KDA_ERR_INVALID_ARG;
@@ -563,6 +621,7 @@ int kda_decode_destroy(kda_handle h)
     int rc = KDA_OK;
     if (cudaStreamSynchronize(h->stream) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     kda::fused_destroy(&h->fused);
+    if (h->pf_ws && cudaFree(h->pf_ws) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     if (h->status_host && cudaFreeHost(h->status_host) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     if (cudaFree(h->scratch_base) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     delete h;

@@ -41,6 +41,19 @@ int simple_launches();
 cudaError_t simple_step_tokens(const Dims &d, int tokens, const kda_weights &w, const void *x, float *state,
                                void *out, int out_dtype, const Scratch &s, cudaStream_t stream);
 
+// Stages of the simple engine, for d.B activation rows (used by the chunked prefill):
+// q, k, v, W_b x, t and z into s; and out = W_o o.
+cudaError_t simple_projections(const Dims &d, const kda_weights &w, const void *x, const Scratch &s, cudaStream_t st);
+cudaError_t simple_out_projection(const Dims &d, const kda_weights &w, const float *o, void *out, int out_dtype,
+                                  cudaStream_t st);
+
+// Chunked form of the recurrence for nseq sequences of T tokens (activations of row b*T + t in
+// s, as simple_projections leaves them): o of every token into s.o, the state advanced by T
+// tokens.  chunk: tokens per chunk (chunk_supported says which).
+bool chunk_supported(int dk, int dv, int chunk);
+size_t chunk_smem_bytes(int dk, int dv, int chunk);
+cudaError_t chunk_state(const Dims &d, int nseq, int T, int chunk, const Scratch &s, float *state, cudaStream_t st);
+
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__
 

@@ -258,10 +258,10 @@ void launch_state_tokens(const Dims &d, int nseq, int T, const Scratch &s, float
     k_state_tokens<DK, DV><<<dim3(d.nh, nseq), DV, 0, st>>>(s.q, s.k, s.v, s.bpre, s.z, state, s.o, d.nh, T);
 }
 
-// The five stages for d.B activation rows; the state stage covers nseq sequences of T
-// tokens each (d.B = nseq * T; T == 1 is the single-token step).
-cudaError_t simple_run(const Dims &d, int nseq, int T, const kda_weights &w, const void *x, float *state,
-                       void *out, int out_dtype, const Scratch &s, cudaStream_t st)
+}  // namespace
+
+// Stages 1-3 for d.B activation rows: q, k, v, W_b x, t = W_a_down x and z = W_a_up t.
+cudaError_t simple_projections(const Dims &d, const kda_weights &w, const void *x, const Scratch &s, cudaStream_t st)
 {
     const int H = d.H, Dk = d.Dk(), Dv = d.Dv();
     const int by = (d.B + kBatchChunk - 1) / kBatchChunk;
@@ -290,6 +290,34 @@ cudaError_t simple_run(const Dims &d, int nseq, int T, const kda_weights &w, con
         GemvJob jz{w.wa_up, s.z, Dk};
         k_gemv_bf16<float><<<dim3((Dk + 7) / 8, by, 1), 256, 0, st>>>(jz, jz, d.r, s.t, d.B);
     }
+    return cudaGetLastError();
+}
+
+// Stage 5 for d.B rows: out = W_o o.
+cudaError_t simple_out_projection(const Dims &d, const kda_weights &w, const float *o, void *out, int out_dtype,
+                                  cudaStream_t st)
+{
+    const int H = d.H, Dv = d.Dv();
+    const int by = (d.B + kBatchChunk - 1) / kBatchChunk;
+    ProjJob jo{w.wo, w.so, nullptr};
+    if (out_dtype == KDA_OUT_BF16)
+        k_proj_fp8<float, __nv_bfloat16><<<dim3((H + 7) / 8, by, 1), 256, 0, st>>>(
+            jo, jo, jo, H, Dv, o, d.B, static_cast<__nv_bfloat16 *>(out));
+    else
+        k_proj_fp8<float, float><<<dim3((H + 7) / 8, by, 1), 256, 0, st>>>(jo, jo, jo, H, Dv, o, d.B,
+                                                                          static_cast<float *>(out));
+    return cudaGetLastError();
+}
+
+namespace {
+
+// The five stages for d.B activation rows; the state stage covers nseq sequences of T
+// tokens each (d.B = nseq * T; T == 1 is the single-token step).
+cudaError_t simple_run(const Dims &d, int nseq, int T, const kda_weights &w, const void *x, float *state,
+                       void *out, int out_dtype, const Scratch &s, cudaStream_t st)
+{
+    cudaError_t e = simple_projections(d, w, x, s, st);
+    if (e != cudaSuccess) return e;
     // 4. state update and readout
     if (T == 1) {
         if (d.dk == 128 && d.dv == 128) launch_state<128, 128>(d, s, state, st);
@@ -303,16 +331,7 @@ cudaError_t simple_run(const Dims &d, int nseq, int T, const kda_weights &w, con
         else launch_state_tokens<64, 128>(d, nseq, T, s, state, st);
     }
     // 5. out = W_o o
-    {
-        ProjJob jo{w.wo, w.so, nullptr};
-        if (out_dtype == KDA_OUT_BF16)
-            k_proj_fp8<float, __nv_bfloat16><<<dim3((H + 7) / 8, by, 1), 256, 0, st>>>(
-                jo, jo, jo, H, Dv, s.o, d.B, static_cast<__nv_bfloat16 *>(out));
-        else
-            k_proj_fp8<float, float><<<dim3((H + 7) / 8, by, 1), 256, 0, st>>>(jo, jo, jo, H, Dv, s.o, d.B,
-                                                                              static_cast<float *>(out));
-    }
-    return cudaGetLastError();
+    return simple_out_projection(d, w, s.o, out, out_dtype, st);
 }
 
 }  // namespace
