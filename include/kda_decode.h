@@ -222,6 +222,42 @@ KDA_API int kda_state_restore(kda_handle h, const void *host_src, float *state, 
  */
 KDA_API int kda_decode_set_launch_overlap(kda_handle h, int on);
 
+/*
+ * Tensor parallelism by heads with the out all-reduce inside the fused kernel.
+ *
+ * The TrnRT story runs decode tensor-parallel and folds each collective that would block the
+ * next kernel into the kernel itself (its third rule).  For this layer half a head split
+ * needs one exchange: rank g of `world` holds the rows of W_q, W_k, W_v, W_a_up and W_b for
+ * its heads, their state, the matching column block of W_o and a whole W_a_down, and its
+ * step forms the partial out = W_o[:, its heads] o; the layer's out is the sum over ranks.
+ * Configured handles do that sum in the step's own kernel: as soon as a block of 32 output
+ * rows is final, each rank stores its partial rows into every rank's exchange region over
+ * peer memory (NVLink), raises that block's flag there (release, system scope), and then
+ * adds the ranks' partials in rank order, so every rank writes the same out bits.  Each
+ * rank's handle is created with its own shard's shape (num_heads = heads per rank).
+ *
+ * kda_tp_configure(h, rank, world, handle_out): allocates this rank's exchange region on
+ *   the handle's device (2 x world x max_batch x hidden fp32 partials and 2 x world x
+ *   hidden / 32 flags; two parities so that a step never overwrites rows a peer may still
+ *   read) and writes its CUDA IPC handle (KDA_TP_HANDLE_BYTES bytes) to handle_out when
+ *   world > 1 (handle_out may be NULL when world = 1).  1 <= world <= 8, 0 <= rank < world.
+ *   Needs the fused engine (KDA_ERR_UNSUPPORTED_SHAPE otherwise); a handle is configured
+ *   once (KDA_ERR_INVALID_ARG on a second call).
+ * kda_tp_set_peer(h, peer, handle): maps rank `peer`'s exchange region from the handle that
+ *   rank's kda_tp_configure wrote (cudaIpcOpenMemHandle; the two devices must have peer
+ *   access).  Steps return KDA_ERR_INVALID_ARG until every peer is mapped.
+ * After configuration every step of the handle (kda_decode_step, kda_decode_step_tokens)
+ *   returns the whole out, and must take the fused engine (KDA_ERR_UNSUPPORTED_SHAPE, with
+ *   nothing enqueued, for a batch it does not cover).  All ranks must issue the same steps
+ *   in the same order: a step's kernel waits (bounded by the handle's timeout) for the
+ *   matching step of every peer.  A timed-out wait leaves the group out of step; destroy
+ *   and recreate the handles of every rank.  The regions are freed (peers unmapped) by
+ *   kda_decode_destroy.
+ */
+#define KDA_TP_HANDLE_BYTES 64
+KDA_API int kda_tp_configure(kda_handle h, int rank, int world, void *handle_out);
+KDA_API int kda_tp_set_peer(kda_handle h, int peer, const void *handle);
+
 /* Waits for the handle's stream; returns the device status of the steps since
  * the last check (KDA_OK or KDA_ERR_DEVICE_TIMEOUT) and clears it. */
 KDA_API int kda_decode_sync(kda_handle h);

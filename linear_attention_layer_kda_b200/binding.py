@@ -34,8 +34,10 @@ EXPORTS = (
     "kda_decode_destroy", "kda_decode_engine", "kda_decode_launches_per_step", "kda_decode_scratch_bytes",
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
     "kda_decode_step_noalloc", "kda_decode_step_tokens", "kda_state_checkpoint", "kda_state_restore",
-    "kda_decode_set_launch_overlap", "kda_decode_tokens_engine", "kda_prefill",
+    "kda_decode_set_launch_overlap", "kda_decode_tokens_engine", "kda_prefill", "kda_tp_configure",
+    "kda_tp_set_peer",
 )
+KDA_TP_HANDLE_BYTES = 64
 KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
 KDA_DEBUG_Q, KDA_DEBUG_K, KDA_DEBUG_V, KDA_DEBUG_BETA_PRE, KDA_DEBUG_T = range(5)
 
@@ -98,6 +100,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_decode_set_launch_overlap": (I, [P, I]),
         "kda_decode_tokens_engine": (I, [P, I, I]),
         "kda_prefill": (I, [P, P, ctypes.POINTER(kda_weights), P, P, I, I, I]),
+        "kda_tp_configure": (I, [P, I, I, P]),
+        "kda_tp_set_peer": (I, [P, I, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -150,6 +154,19 @@ def kda_decode_step_host(h: int, x_host: int, w: kda_weights, state: int, out_ho
 
 def kda_decode_set_launch_overlap(h: int, on: bool) -> None:
     _check(load().kda_decode_set_launch_overlap(h, 1 if on else 0), "kda_decode_set_launch_overlap", h)
+
+
+def kda_tp_configure(h: int, rank: int, world: int) -> bytes:
+    buf = ctypes.create_string_buffer(KDA_TP_HANDLE_BYTES)
+    _check(load().kda_tp_configure(h, rank, world, buf), "kda_tp_configure", h)
+    return buf.raw
+
+
+def kda_tp_set_peer(h: int, peer: int, handle: bytes) -> None:
+    if len(handle) != KDA_TP_HANDLE_BYTES:
+        raise ValueError(f"an exchange handle has {KDA_TP_HANDLE_BYTES} bytes, got {len(handle)}")
+    buf = ctypes.create_string_buffer(handle, KDA_TP_HANDLE_BYTES)
+    _check(load().kda_tp_set_peer(h, peer, buf), "kda_tp_set_peer", h)
 
 
 def kda_decode_sync(h: int) -> None:
@@ -315,6 +332,13 @@ class KdaDecoder:
         self._bind_stream()
         kda_decode_debug_copy(self.h, which, t.data_ptr(), t.numel() * 4)
         return t
+
+    def tp_configure(self, rank: int, world: int) -> bytes:
+        """Exchange region of rank `rank` of `world`; returns its IPC handle for the peers."""
+        return kda_tp_configure(self.h, rank, world)
+
+    def tp_set_peer(self, peer: int, handle: bytes) -> None:
+        kda_tp_set_peer(self.h, peer, handle)
 
     def engine(self, batch: int) -> int:
         return kda_decode_engine(self.h, batch)

@@ -165,9 +165,20 @@ int check_usable(kda_handle h)
     return fail(h, KDA_ERR_DEVICE_TIMEOUT, "handle unusable: an aborted step did not drain its copies in flight");
 }
 
+// A tensor-parallel handle runs only fused steps, and only once every peer is mapped.
+int check_tp(kda_handle h, int engine)
+{
+    if (!h->fused.tp_world) return KDA_OK;
+    if (engine != KDA_ENGINE_FUSED)
+        return fail(h, KDA_ERR_UNSUPPORTED_SHAPE, "tensor parallelism needs the fused engine for this step");
+    if (!h->fused.tp_ready) return fail(h, KDA_ERR_INVALID_ARG, "tensor-parallel peers are not all mapped");
+    return KDA_OK;
+}
+
 int enqueue_step(kda_handle h, const void *x, const kda_weights *w, float *state, void *out, int batch)
 {
     const kda::Dims d = dims_of(h->cfg, batch);
+    if (int rc = check_tp(h, pick_engine(h, batch))) return rc;
     cudaError_t e;
     if (pick_engine(h, batch) == KDA_ENGINE_FUSED)
         e = kda::fused_step(d, 1, *w, x, state, out, h->cfg.out_dtype, h->fused, h->s, h->status, h->stream);
@@ -404,6 +415,55 @@ int kda_decode_set_stream(kda_handle h, void *stream)
     return KDA_OK;
 }
 
+int kda_tp_configure(kda_handle h, int rank, int world, void *ipc_handle_out)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    kda::FusedState &fs = h->fused;
+    if (world < 1 || world > 8 || rank < 0 || rank >= world)
+        return fail(h, KDA_ERR_INVALID_ARG, "need 1 <= world <= 8 and 0 <= rank < world");
+    if (fs.tp_world) return fail(h, KDA_ERR_INVALID_ARG, "tensor parallelism is already configured");
+    if (!fs.bytes) return fail(h, KDA_ERR_UNSUPPORTED_SHAPE, "the in-kernel reduction needs the fused engine");
+    const size_t H = (size_t)h->cfg.hidden, bmax = (size_t)h->cfg.max_batch;
+    fs.tp_slot_bytes = 2 * world * bmax * H * 4;
+    const size_t bytes = fs.tp_slot_bytes + 2 * (size_t)world * (H / 32) * 4;
+    void *region = nullptr;
+    cudaError_t e = cudaMalloc(&region, bytes);
+    if (e == cudaSuccess) e = cudaMemset(region, 0, bytes);
+    cudaIpcMemHandle_t ipc;
+    if (e == cudaSuccess && world > 1) e = cudaIpcGetMemHandle(&ipc, region);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        if (region) cudaFree(region);
+        return cuda_fail(h, e, "exchange region");
+    }
+    if (ipc_handle_out && world > 1) memcpy(ipc_handle_out, &ipc, sizeof ipc);
+    fs.tp_world = world;
+    fs.tp_rank = rank;
+    fs.tp_bmax = (int)bmax;
+    fs.tp_region[rank] = region;
+    fs.tp_ready = world == 1;
+    return KDA_OK;
+}
+
+int kda_tp_set_peer(kda_handle h, int peer, const void *ipc_handle)
+{
+    if (!h || !ipc_handle) return KDA_ERR_INVALID_ARG;
+    kda::FusedState &fs = h->fused;
+    if (!fs.tp_world) return fail(h, KDA_ERR_INVALID_ARG, "tensor parallelism is not configured");
+    if (peer < 0 || peer >= fs.tp_world || peer == fs.tp_rank) return fail(h, KDA_ERR_INVALID_ARG, "bad peer rank");
+    if (fs.tp_region[peer]) return fail(h, KDA_ERR_INVALID_ARG, "peer already mapped");
+    cudaIpcMemHandle_t ipc;
+    memcpy(&ipc, ipc_handle, sizeof ipc);
+    void *p = nullptr;
+    const cudaError_t e = cudaIpcOpenMemHandle(&p, ipc, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(h, e, "mapping a peer's exchange region");
+    fs.tp_region[peer] = p;
+    bool all = true;
+    for (int r = 0; r < fs.tp_world; ++r) all = all && fs.tp_region[r];
+    fs.tp_ready = all;
+    return KDA_OK;
+}
+
 int kda_decode_set_launch_overlap(kda_handle h, int on)
 {
     if (!h) return KDA_ERR_INVALID_ARG;
@@ -488,6 +548,7 @@ int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, fl
         return fail(h, KDA_ERR_INVALID_ARG, "state_inout overlaps x or out");
     rc = take_device_status(h);
     if (rc) return rc;
+    if (int rc1 = check_tp(h, tokens_engine(h, batch, tokens))) return rc1;
     cudaError_t e;
     if (tokens_engine(h, batch, tokens) == KDA_ENGINE_FUSED)
         e = kda::fused_step(dims_of(c, batch * tokens), tokens, *w, x, state_inout, out, c.out_dtype, h->fused, h->s,
@@ -622,6 +683,12 @@ int kda_decode_destroy(kda_handle h)
     if (cudaStreamSynchronize(h->stream) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     kda::fused_destroy(&h->fused);
     if (h->pf_ws && cudaFree(h->pf_ws) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    for (int r = 0; r < h->fused.tp_world; ++r) {
+        void *p = h->fused.tp_region[r];
+        if (!p) continue;
+        const cudaError_t e = r == h->fused.tp_rank ? cudaFree(p) : cudaIpcCloseMemHandle(p);
+        if (e != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    }
     if (h->status_host && cudaFreeHost(h->status_host) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     if (cudaFree(h->scratch_base) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     delete h;

@@ -88,12 +88,12 @@ constexpr int kSegBars = 32;          // segment hand-off barriers (epilogue -> 
 #endif
 enum TraceSlot {
     TR_START = 0, TR_XREADY, TR_FIRST_MMA, TR_QKV_DONE, TR_EPI_DONE, TR_XQ_DONE, TR_GATES_DONE,
-    TR_UNIT0 = 7,  /* 3 stamps per unit: claimed, inputs ready, done; 2 units */
-    TR_UNIT_SUMS = 13, /* units 0, 1: partial sums loaded */ TR_UNIT_HAND = 15, /* units 0, 1: o handed off */
-    TR_UNIT_ITEMS = 17, /* unit 0: all partial sums in shared memory */ TR_UNIT_O = 18, /* unit 0: o computed */
+    TR_UNIT0 = 7,  /* units 0, 1: claimed, (unused), done */
+    TR_UNIT_HAND = 15, /* units 0, 1: o handed off */
     TR_PUB0 = 25, /* publisher: release of segment k issued and done, k < 7 */
     TR_O_WAIT0 = 19, TR_O_READY0, TR_O_READY_LAST, TR_END, TR_LAST_REDUCE_START, TR_LAST_REDUCE_END,
-    TR_TILE_TMA = 32, TR_TILE_MMA = 64, TR_TILE_EPI = 96, TR_TILE_TMA_RET = 128, TR_TILE_ACT = 160 /* per tile i < 32 */
+    TR_TILE_TMA = 32, TR_TILE_MMA = 64, TR_TILE_EPI = 96, TR_USUB = 128, /* 16 stamps per state unit, units < 2 */
+    TR_TILE_ACT = 160 /* per tile i < 32 */
 };
 
 // counters (uint32, monotonic across steps; targets are multiples of the step count)
@@ -112,17 +112,21 @@ constexpr int ST_CODE = 0, ST_WHERE = 1, ST_DRAIN = 2;
 constexpr int kOHand = 8;  // o-block hand-off barriers (state unit -> o publisher), reused mod 8
 
 constexpr int kMaxT = 8;  // tokens per sequence in one multi-token step
+constexpr int kMaxTp = 8;  // ranks of a tensor-parallel group
 
-struct __align__(16) VecSmem {
+// NT: tokens per unit (1, or kMaxT in the multi-token kernels).
+template <int NT>
+struct __align__(16) VecSmemT {
+    static constexpr int NA = NT < 2 ? 2 : NT;  // gate slots (one token: the current and the next unit)
     uint64_t ohand[kOHand];        // unit k's o planes are stored (arrival of vector warp 0)
     int opub;                      // units whose o block the o publisher has released
     int pad_[3];
-    float q[kMaxT][256], k[kMaxT][256];  // per token and head of the unit: q, k^ (heads_per_unit * dk)
-    float a[kMaxT][256];           // alpha per token (one token: slots of the current and next unit)
-    float v[kMaxT][128];           // per token and virtual column of the unit
+    float q[NT][256], k[NT][256];  // per token and head of the unit: q, k^ (heads_per_unit * dk)
+    float a[NA][256];              // alpha per gate slot
+    float v[NT][128];              // per token and virtual column of the unit
     float u[128], o[128];
     float red_w[8][128], red_p[8][128];  // adjacent: also the t rows of token_gates
-    float beta[kMaxT][2], kq[kMaxT][2], inv[kMaxT][2];
+    float beta[NA][2], kq[NT][2], inv[NT][2];
     int unit, ok, fail;
 };
 
@@ -153,6 +157,12 @@ struct FusedParams {
     uint32_t epoch, t_xq, t_gate, t_o;
     uint64_t timeout_ns;
     int out_bf16, stages, a_bytes, w_bytes, nacc, cols, skip_gate_release, early_tiles;
+    // tensor parallelism by heads (tp_world > 0): this rank's partial out goes to every rank's
+    // exchange slots [parity][src][tp_bmax][H] fp32 and their flags [parity][src][H / 32]
+    int tp_world, tp_rank, tp_bmax;
+    uint32_t tp_epoch;
+    float *tp_slots[kMaxTp];
+    uint32_t *tp_flags[kMaxTp];
 };
 
 // Floats per partial-sum slot: [pair][BP][N <= 256]; pair 1 only for the o planes 2 and 3.
@@ -239,6 +249,34 @@ __device__ bool wait_count(const uint32_t *p, uint32_t target, const Ctl &c, int
             return false;
         }
     }
+}
+
+// Bounded wait until a flag that another GPU writes equals `want` (system-scope acquire).
+__device__ bool wait_flag_sys(const uint32_t *p, uint32_t want, const Ctl &c, int where)
+{
+    auto ld = [](const uint32_t *q) {
+        uint32_t v;
+        asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(q) : "memory");
+        return v;
+    };
+    if (ld(p) == want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t next = t0 + 20000;
+    for (;;) {
+        __nanosleep(64);
+        if (ld(p) == want) return true;
+        const uint64_t now = globaltimer_ns();
+        if (poll_abort(c, now, next)) return false;
+        if (now - t0 > c.P.timeout_ns) {
+            raise_abort(c, where);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void st_release_sys(uint32_t *p, uint32_t v)
+{
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ int rg_key(const FusedParams &P, int mat, int rg)
@@ -387,8 +425,8 @@ __device__ void quantize_x(const FusedParams &P, int gw, int ngw, int lane)
 
 // Gate rows (W_b and W_a_down, bf16): one row per CTA at a time, its K range split over the
 // eight vector warps, partial sums added in warp order through shared memory.
-template <int BP>
-__device__ void gate_rows(const FusedParams &P, VecSmem *vs, int vt)
+template <int BP, class VS>
+__device__ void gate_rows(const FusedParams &P, VS *vs, int vt)
 {
     const int vw = vt >> 5, lane = vt & 31;
     const int rows = P.nh + P.r;
@@ -448,8 +486,8 @@ __device__ void gate_rows(const FusedParams &P, VecSmem *vs, int vt)
 // Gates of state unit u (sequence u % B, o K-block u / B) into slot `slot`: beta of its
 // heads and alpha = exp(-softplus(z)) = 1 / (1 + e^z), z = W_a_up[row] . t, of its rows,
 // computed by vector threads [t0, t0 + nt).  t and W_b x must be final (C_GATE acquired).
-template <int DK>
-__device__ void unit_gates(const FusedParams &P, VecSmem *vs, int u, int slot, int vt, int t0, int nt)
+template <int DK, class VS>
+__device__ void unit_gates(const FusedParams &P, VS *vs, int u, int slot, int vt, int t0, int nt)
 {
     const int b = u % P.Bs, kb = u / P.Bs, hpu = 128 / P.dv, h0 = kb * hpu;
     const int me = vt - t0;
@@ -487,8 +525,8 @@ __device__ void unit_gates(const FusedParams &P, VecSmem *vs, int u, int slot, i
 // Gates of this CTA's first two units (u1 < 0: none) into slots 0 and 1, by all 256 vector
 // threads with every load issued in one batch: t of the two sequences into shared memory,
 // beta, and one W_a_up row per thread and unit.  t and W_b x must be final.
-template <int DK>
-__device__ void first_gates(const FusedParams &P, VecSmem *vs, int u0, int u1, int vt)
+template <int DK, class VS>
+__device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt)
 {
     const int hpu = 128 / P.dv, rows = hpu * DK, r4 = P.r / 4;
     const int us[2] = {u0, u1};
@@ -539,8 +577,8 @@ __device__ void first_gates(const FusedParams &P, VecSmem *vs, int u0, int u1, i
 // Gates of every token of a multi-token unit (sequence bs, o K-block kb): alpha into a[t],
 // beta into beta[t].  Each thread loads one W_a_up row once and dots it with the T rows of t
 // (staged in shared memory).  t and W_b x must be final.
-template <int DK>
-__device__ void token_gates(const FusedParams &P, VecSmem *vs, int bs, int kb, int vt)
+template <int DK, class VS>
+__device__ void token_gates(const FusedParams &P, VS *vs, int bs, int kb, int vt)
 {
     const int T = P.T, hpu = 128 / P.dv, rows = hpu * DK, h0 = kb * hpu, r4 = P.r / 4;
     float *ts = &vs->red_w[0][0];  // [T][r], T * r <= 2048 (red_w and red_p)
@@ -600,8 +638,8 @@ __device__ void token_gates(const FusedParams &P, VecSmem *vs, int bs, int kb, i
 // its gates are in slot nu & 1 and, while a few threads wait for the unit's q/k/v, the others
 // compute the gates of this CTA's next unit (next_u >= 0) into the other slot; with several
 // tokens every token's gates are computed here.
-template <int BP, int DK, bool MT>
-__device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int u, int next_u, int vt, int nu)
+template <int BP, int DK, bool MT, class VS>
+__device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, int next_u, int vt, int nu)
 {
     constexpr ActGeo G = act_geo(BP);
     const int T = MT ? P.T : 1, bs = u % P.Bs, kb = u / P.Bs, slot = nu & 1;
@@ -620,6 +658,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 
     if (vt == 0) vs->fail = 0;
     named_bar(2, 256);
+    if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu);
     // then the heads' q, k, v: wait for every segment of their row groups (one thread per
     // counter, so the round trips overlap), add the partials
     {
@@ -633,7 +672,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         if (!MT && next_u >= 0 && nu >= 1) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
     }
     named_bar(2, 256);
-    if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu + 1);
+    if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu + 1);
     if (vs->fail) return false;
     if (MT) {
         token_gates<DK>(P, vs, bs, kb, vt);
@@ -664,7 +703,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
             }
             float val[2];
             sum_segs2<BP>(P, key, off, has, val);
-            if (vt == 0 && nu < 2 && it0 == 0) KDA_TR(P, TR_UNIT_SUMS + nu);
+            if (vt == 0 && nu < 2 && it0 == 0) KDA_TR(P, TR_USUB + 16 * nu + 2);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int it = it0 + vt + 256 * j, t = it / per, i = it % per, row = bs * T + t;
@@ -682,7 +721,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         }
     }
     named_bar(2, 256);
-    if (vt == 0 && nu == 0) KDA_TR(P, TR_UNIT_ITEMS);
+    if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu + 3);
     // ||k|| and k.q per token and head (one warp per pair)
     for (int pr = vw; pr < T * hpu; pr += 8) {
         const int t = pr / hpu, hd = pr % hpu;
@@ -703,7 +742,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
     named_bar(2, 256);
     for (int i = vt; i < T * nqk; i += 256) vs->k[i / nqk][i % nqk] *= vs->inv[i / nqk][(i % nqk) / DK];
     named_bar(2, 256);
-
+    if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu + 4);
     for (int t = 0; t < T; ++t) {
         const float *al = vs->a[MT ? t : slot];
         const float *kt = vs->k[t], *qt = vs->q[t];
@@ -722,6 +761,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
         *reinterpret_cast<float4 *>(&vs->red_w[vw][vc]) = pw;
         *reinterpret_cast<float4 *>(&vs->red_p[vw][vc]) = pp;
         named_bar(2, 256);
+        if (vt == 0 && nu < 2 && t == 0) KDA_TR(P, TR_USUB + 16 * nu + 9);
         if (vt < 128) {
             float w = 0.f, p = 0.f;
 #pragma unroll
@@ -735,7 +775,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
             vs->o[vt] = fmaf(uu, vs->kq[t][hx], p);
         }
         named_bar(2, 256);
-        if (vt == 0 && nu == 0 && t == 0) KDA_TR(P, TR_UNIT_O);
+        if (vt == 0 && nu < 2 && t == 0) KDA_TR(P, TR_USUB + 16 * nu + 5);
         // o of row bs*T + t -> four E4M3 planes with one power-of-two scale for the K-block
         if (vw == 0) {
             const int row = bs * T + t;
@@ -750,6 +790,7 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
             if (lane == 0)
                 *reinterpret_cast<float *>(P.oq + (size_t)(G.rso + row / 32) * Dv + (size_t)kb * 128 + (row % 32) * 4) = sc;
             fence_proxy_async_global();
+            if (lane == 0 && nu < 2 && t == 0) KDA_TR(P, TR_USUB + 16 * nu + 6);
         }
         // S' = S~ + k^ u^T (kept in registers for the next token)
         const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
@@ -776,12 +817,14 @@ __device__ bool state_unit(const FusedParams &P, VecSmem *vs, const Ctl &c, int 
 #pragma unroll
     for (int r = 0; r < RPW; ++r) st_stream_f4(S + (size_t)(vw * RPW + r) * dv, s[r]);
     named_bar(2, 256);
+    if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu + 7);
     return true;
 }
 
 // Warp 1, lane 0: releases the o blocks of this CTA's state units, in unit order, once vector
 // warp 0 has stored their planes.
-__device__ void o_publisher(const FusedParams &P, VecSmem *vs, const Ctl &c)
+template <class VS>
+__device__ void o_publisher(const FusedParams &P, VS *vs, const Ctl &c)
 {
     const int units = P.Bs * P.nKBo;
     for (int k = 0, u = blockIdx.x; u < units; ++k, u += gridDim.x) {
@@ -802,8 +845,8 @@ __device__ void prefetch_unit_state(const FusedParams &P, int u)
         bulk_prefetch_l2_hint(p + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
 }
 
-template <int BP, int DK, bool MT>
-__device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
+template <int BP, int DK, bool MT, class VS>
+__device__ void vector_role(const FusedParams &P, VS *vs, const Ctl &c)
 {
     constexpr ActGeo G = act_geo(BP);
     const int vt = threadIdx.x - 256, vw = vt >> 5, lane = vt & 31;
@@ -827,18 +870,25 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
         if (vt == 0) vs->unit = should_stop(c) ? 1 : 0;
         named_bar(2, 256);
         if (vs->unit) return;
-        if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu);
+        if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu);
         const int next = u + (int)gridDim.x < units ? u + (int)gridDim.x : -1;
         if (vt == 0 && next >= 0) prefetch_unit_state(P, next);  // its state streams in meanwhile
         if (!state_unit<BP, DK, MT>(P, vs, c, u, next, vt, nu)) return;
-        if (vt == 0 && nu < 4) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
+        if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
     }
-    // out = sum of the W_o partials (both plane pairs): items of 32 output rows
-    for (int item = blockIdx.x; item < P.H / 32; item += gridDim.x) {
+    // out = sum of the W_o partials (both plane pairs): items of 32 output rows.  With tensor
+    // parallelism the sum is this rank's partial out: it is pushed to every rank's exchange
+    // slot (peer stores over NVLink), the item's flag is raised in every rank, and each rank
+    // then adds the ranks' partials in rank order (the same bits everywhere).
+    const int nitems = P.H / 32, par = (int)(P.tp_epoch & 1u);
+    const size_t slot_sz = (size_t)P.tp_world * P.tp_bmax * P.H;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
         const int grow0 = item * 32, rg = grow0 / G.no, key = 2 * P.nRGq + P.nRGv + rg;
+        if (vt == 0 && item == (int)blockIdx.x) KDA_TR(P, TR_LAST_REDUCE_START);
         if (vt == 0) vs->ok = wait_rb(P, key, c, 12);
         named_bar(2, 256);
         if (!vs->ok) return;
+        if (vt == 0 && item == (int)blockIdx.x) KDA_TR(P, TR_O_WAIT0);
         const int grow = grow0 + lane, n = grow % G.no;
         for (int b = vw; b < P.B; b += 8) {
             const int kk[2] = {key, key}, off[2] = {b * G.no + n, (BP + b) * G.no + n};
@@ -846,10 +896,37 @@ __device__ void vector_role(const FusedParams &P, VecSmem *vs, const Ctl &c)
             float val[2];
             sum_segs2<BP>(P, kk, off, has, val);
             const float v = val[0] + val[1];
+            if (P.tp_world > 0) {
+                const size_t o = par * slot_sz + ((size_t)P.tp_rank * P.tp_bmax + b) * P.H + grow;
+                for (int r = 0; r < P.tp_world; ++r) P.tp_slots[r][o] = v;
+            } else if (P.out_bf16) {
+                static_cast<__nv_bfloat16 *>(P.out)[(size_t)b * P.H + grow] = __float2bfloat16_rn(v);
+            } else {
+                static_cast<float *>(P.out)[(size_t)b * P.H + grow] = v;
+            }
+        }
+        if (P.tp_world > 0) __threadfence_system();  // the pushed rows before the flags
+        named_bar(2, 256);
+        if (P.tp_world > 0 && vt < P.tp_world)
+            st_release_sys(P.tp_flags[vt] + ((size_t)par * P.tp_world + P.tp_rank) * nitems + item, P.tp_epoch);
+        if (vt == 0 && item == (int)blockIdx.x) KDA_TR(P, TR_LAST_REDUCE_END);
+    }
+    if (P.tp_world == 0) return;
+    const float *mine = P.tp_slots[P.tp_rank] + par * slot_sz;
+    const uint32_t *flags = P.tp_flags[P.tp_rank] + (size_t)par * P.tp_world * nitems;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        if (vt == 0) vs->fail = 0;
+        named_bar(2, 256);
+        if (vt < P.tp_world && !wait_flag_sys(flags + (size_t)vt * nitems + item, P.tp_epoch, c, 15)) vs->fail = 1;
+        named_bar(2, 256);
+        if (vs->fail) return;
+        const int grow = item * 32 + lane;
+        for (int b = vw; b < P.B; b += 8) {
+            float v = 0.f;
+            for (int r = 0; r < P.tp_world; ++r) v += __ldcv(mine + ((size_t)r * P.tp_bmax + b) * P.H + grow);
             if (P.out_bf16) static_cast<__nv_bfloat16 *>(P.out)[(size_t)b * P.H + grow] = __float2bfloat16_rn(v);
             else static_cast<float *>(P.out)[(size_t)b * P.H + grow] = v;
         }
-        named_bar(2, 256);
     }
 }
 
@@ -1219,8 +1296,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     R.segdone = bars + 3 * kMaxStages + kMaxAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kMaxStages + kMaxAcc + kSegBars);
     volatile int *sh_abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    VecSmem *vs = reinterpret_cast<VecSmem *>(bars + 3 * kMaxStages + kMaxAcc + kSegBars + 2);
-    TileEntry *stiles = reinterpret_cast<TileEntry *>(reinterpret_cast<uint8_t *>(vs) + sizeof(VecSmem));
+    using VS = VecSmemT<MT ? kMaxT : 1>;
+    VS *vs = reinterpret_cast<VS *>(bars + 3 * kMaxStages + kMaxAcc + kSegBars + 2);
+    TileEntry *stiles = reinterpret_cast<TileEntry *>(reinterpret_cast<uint8_t *>(vs) + sizeof(VS));
 
     // this CTA's tile list -> shared memory (read by every role, once per tile)
     const uint32_t t_begin = P.cta_off[blockIdx.x];
@@ -1397,10 +1475,12 @@ void *pick_kernel_t(int BP, int DK)
 }
 void *pick_kernel(int BP, int DK, bool multi) { return multi ? pick_kernel_t<true>(BP, DK) : pick_kernel_t<false>(BP, DK); }
 
-size_t fixed_smem_bytes(int max_tiles)
+// Shared memory past the ring: barriers, the vector warps' area, the tile list (+ the 1 KB
+// alignment slack of the dynamic allocation).
+size_t fixed_smem_bytes(int max_tiles, bool multi)
 {
-    return 1024 /*alignment slack*/ + (3 * kMaxStages + kMaxAcc + kSegBars + 2) * 8 + sizeof(VecSmem) +
-           (size_t)max_tiles * sizeof(TileEntry);
+    return 1024 /*alignment slack*/ + (3 * kMaxStages + kMaxAcc + kSegBars + 2) * 8 +
+           (multi ? sizeof(VecSmemT<kMaxT>) : sizeof(VecSmemT<1>)) + (size_t)max_tiles * sizeof(TileEntry);
 }
 
 constexpr size_t kSmemBudget = 227 * 1024;
@@ -1421,7 +1501,7 @@ bool plan_classes(const Dims &dmax, int num_ctas, int bpm, std::vector<ClassPlan
         fused_build_schedule(dmax, num_ctas, g, &cp.tiles, &cp.off, &cp.nseg, &cp.rbinfo);
         for (int c = 0; c < num_ctas; ++c) cp.max_tiles = std::max(cp.max_tiles, (int)(cp.off[c + 1] - cp.off[c]));
         if (cp.max_tiles > kMaxTilesPerCta) return false;
-        if (fixed_smem_bytes(cp.max_tiles) + 2 * stage_bytes_for(BP) > kSmemBudget) return false;
+        if (fixed_smem_bytes(cp.max_tiles, true) + 2 * stage_bytes_for(BP) > kSmemBudget) return false;
         cp.keys = row_group_keys(dmax, g);
         plans->push_back(std::move(cp));
     }
@@ -1552,7 +1632,8 @@ cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const vo
     if (!fs.uploaded) return cudaErrorNotReady;
     if (tokens < 1 || tokens > kMaxT || d.B % tokens) return cudaErrorNotSupported;
     const int BP = bp_for(d.B), cls = class_of(BP);
-    void *kern = pick_kernel(BP, d.dk, tokens > 1);
+    const bool multi = tokens > 1;
+    void *kern = pick_kernel(BP, d.dk, multi);
     if (!kern || cls >= fs.nclass) return cudaErrorNotSupported;
     const ActGeo g = act_geo(BP);
     const SchedGeo sg = fused_sched_geo(d, BP);
@@ -1658,12 +1739,23 @@ cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const vo
     P.timeout_ns = fs.timeout_ns;
     P.out_bf16 = out_dtype == KDA_OUT_BF16;
     P.skip_gate_release = fs.debug_skip_gate_release;
+    if (fs.tp_world > 0) {
+        if (!fs.tp_ready) return cudaErrorNotReady;
+        P.tp_world = fs.tp_world;
+        P.tp_rank = fs.tp_rank;
+        P.tp_bmax = fs.tp_bmax;
+        P.tp_epoch = fs.tp_epoch + 1;
+        for (int r = 0; r < fs.tp_world; ++r) {
+            P.tp_slots[r] = static_cast<float *>(fs.tp_region[r]);
+            P.tp_flags[r] = reinterpret_cast<uint32_t *>(static_cast<char *>(fs.tp_region[r]) + fs.tp_slot_bytes);
+        }
+    }
     P.a_bytes = (int)a_bytes_for(BP);
     P.w_bytes = (int)w_bytes_for(BP);
     P.cols = tmem_cols_for(BP);
     P.nacc = std::min(kMaxAcc, kTmemCols / P.cols);
     const size_t sbytes = stage_bytes_for(BP);
-    const size_t fixed = fixed_smem_bytes(fs.max_tiles_per_cta[cls]);
+    const size_t fixed = fixed_smem_bytes(fs.max_tiles_per_cta[cls], multi);
     if (fixed + 2 * sbytes > kSmemBudget) return cudaErrorNotSupported;
     int stages = (int)std::min<size_t>(kMaxStagesDefault, (kSmemBudget - fixed) / sbytes);
     if (fs.stages_override > 0)
@@ -1707,6 +1799,7 @@ cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const vo
     cudaError_t e = cudaLaunchKernelExC(&cfg, kern, args);
     if (e != cudaSuccess) return e;
     fs.last_class = cls;
+    if (fs.tp_world > 0) fs.tp_epoch += 1;
     fs.epoch = epoch;
     fs.cum_b += (uint32_t)d.B;
     fs.cum_s += (uint32_t)P.Bs;

@@ -118,6 +118,12 @@ struct FusedState {
     bool amap_ok[4] = {};
     // counter offsets
     int off_oready = 0, off_rb = 0;
+    // tensor parallelism by heads: exchange regions of the group's ranks (slots, then flags)
+    int tp_world = 0, tp_rank = 0, tp_bmax = 0;
+    bool tp_ready = false;          // every rank's region is mapped
+    uint32_t tp_epoch = 0;          // fused steps run in the group (never reset)
+    void *tp_region[8] = {};        // [rank]: slots [2][world][bmax][H] fp32, flags [2][world][H/32]
+    size_t tp_slot_bytes = 0;
 };
 
 bool fused_supports(const Dims &d, int num_sms);

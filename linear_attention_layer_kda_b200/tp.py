@@ -7,9 +7,9 @@ exchange: rank g owns heads [g*nh/G, (g+1)*nh/G) -- the rows of W_q, W_k, W_v, W
 W_b for them, those heads' state, and the matching column block of W_o -- and computes a
 partial out = W_o[:, its columns] o_its_heads.  W_a_down is small and replicated (every
 rank forms t = W_a_down x).  The job's out is the sum of the partials over ranks: one
-all-reduce of B x H fp32 per step, done here with torch.distributed (NCCL on GPUs).
-
-Host-side sharding only: each rank then runs the ordinary single-GPU step on its shard.
+all-reduce of B x H fp32 per step.  By default that sum runs inside the fused kernel over
+peer memory (kda_tp_configure / kda_tp_set_peer); torch.distributed.all_reduce (NCCL on
+GPUs) is the other choice.
 """
 from __future__ import annotations
 
@@ -61,28 +61,76 @@ def shard_inputs(inp: KdaInputs, rank: int, world: int) -> KdaInputs:
     )
 
 
-class TensorParallelDecoder:
-    """One rank of a head-parallel decode step: the local step, then a sum of out over ranks.
+def exchange_handles(dec, rank: int, world: int, group=None) -> None:
+    """Connects the exchange regions of a head-parallel group (every rank calls it, in order).
 
-    `group` is a torch.distributed process group (NCCL for GPUs); every rank calls step()
-    the same number of times, in the same order.
+    Each rank configures its handle (an exchange region on its GPU), the ranks trade the
+    regions' IPC handles with all_gather_object, and each maps its peers' regions.  A rank
+    whose configuration fails sends None instead of a handle; then every rank raises, so no
+    rank is left waiting in a later step for a peer that will never run one.
+    """
+    import torch.distributed as dist
+    err = None
+    try:
+        mine = dec.tp_configure(rank, world)
+    except Exception as e:  # noqa: BLE001 -- reported to every rank below
+        mine, err = None, e
+    handles = [None] * world
+    if world > 1:
+        dist.all_gather_object(handles, mine, group=group)
+    else:
+        handles[0] = mine
+    bad = [r for r, h in enumerate(handles) if h is None]
+    if bad:
+        raise RuntimeError(f"tensor-parallel exchange regions failed on ranks {bad}") from err
+    for peer, h in enumerate(handles):
+        if peer != rank:
+            dec.tp_set_peer(peer, h)
+
+
+class TensorParallelDecoder:
+    """One rank of a head-parallel decode step whose out is the sum over ranks.
+
+    reduce = "fused" (the default): the sum runs inside the step's own kernel over peer
+    memory (kda_tp_configure); every step must take the fused engine.  reduce = "nccl": the
+    local step, then torch.distributed.all_reduce of out (any engine, any backend).
+    `group` is a torch.distributed process group; every rank calls step() the same number of
+    times, in the same order.
     """
 
-    def __init__(self, shard: KdaInputs, max_batch: int, group=None):
+    def __init__(self, shard: KdaInputs, max_batch: int, group=None, reduce: str = "fused", out_dtype=None):
         import torch
         import torch.distributed as dist
 
         from . import binding
+        if reduce not in ("fused", "nccl"):
+            raise ValueError(f"reduce must be 'fused' or 'nccl', got {reduce!r}")
         s = shard.shape
-        self.dec = binding.KdaDecoder(s.hidden, s.num_heads, s.head_dk, s.head_dv, s.alpha_rank, max_batch)
+        kw = {} if out_dtype is None else {"out_dtype": out_dtype}
+        self.dec = binding.KdaDecoder(s.hidden, s.num_heads, s.head_dk, s.head_dv, s.alpha_rank, max_batch, **kw)
         self.group = group
+        self.reduce = reduce
         self._dist = dist
         self._torch = torch
+        if reduce == "fused":
+            rank = dist.get_rank(group) if dist.is_initialized() else 0
+            world = dist.get_world_size(group) if dist.is_initialized() else 1
+            try:
+                exchange_handles(self.dec, rank, world, group)
+            except Exception:
+                self.dec.close()
+                raise
 
-    def step(self, x, weights, state_shard, out) -> None:
-        """out (fp32 [B, H]) becomes the whole layer half's output on every rank."""
-        self.dec.step(x, weights, state_shard, out)
-        self._dist.all_reduce(out, op=self._dist.ReduceOp.SUM, group=self.group)
+    def step(self, x, weights, state_shard, out, batch=None) -> None:
+        """out ([B, H]) becomes the whole layer half's output on every rank."""
+        self.dec.step(x, weights, state_shard, out, batch)
+        if self.reduce == "nccl":
+            self._dist.all_reduce(out, op=self._dist.ReduceOp.SUM, group=self.group)
+
+    def step_tokens(self, x, weights, state_shard, out, batch: int, tokens: int) -> None:
+        self.dec.step_tokens(x, weights, state_shard, out, batch, tokens)
+        if self.reduce == "nccl":
+            self._dist.all_reduce(out, op=self._dist.ReduceOp.SUM, group=self.group)
 
     def sync(self) -> None:
         self.dec.sync()

@@ -92,3 +92,59 @@ def test_shard_layout():
         tp.head_range(32, 0, 3)
     with pytest.raises(ValueError):  # 1 head of 64 per rank: not a whole 128-wide block
         tp.check_shardable(I.CONFIGS[0], 2)
+
+
+class _FakeHandle:
+    """Stands in for a KdaDecoder's tensor-parallel calls (no GPU): records what it was given."""
+
+    def __init__(self, rank, fail_rank=None):
+        self.rank, self.fail_rank = rank, fail_rank
+        self.configured, self.peers = None, {}
+
+    def tp_configure(self, rank, world):
+        if rank == self.fail_rank:
+            raise RuntimeError("no exchange region")
+        self.configured = (rank, world)
+        return bytes([rank + 1]) * 64
+
+    def tp_set_peer(self, peer, handle):
+        self.peers[peer] = handle
+
+
+def _exchange_main(rank, world, port, outdir, fail_rank):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from linear_attention_layer_kda_b200 import tp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        fake = _FakeHandle(rank, fail_rank)
+        try:
+            tp.exchange_handles(fake, rank, world)
+            result = {"configured": fake.configured, "peers": {p: h[0] for p, h in fake.peers.items()}}
+        except RuntimeError as e:
+            result = {"error": str(e), "peers": {p: h[0] for p, h in fake.peers.items()}}
+        np.save(os.path.join(outdir, f"x{rank}.npy"), np.array([repr(result)]))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,fail_rank", [(2, None), (3, None), (3, 1)])
+def test_exchange_handles_over_gloo(tmp_path, world, fail_rank):
+    """Every rank maps every other rank's region with that rank's handle; a failed rank fails all."""
+    import ast
+    mp.start_processes(_exchange_main, args=(world, _free_port(), str(tmp_path), fail_rank), nprocs=world,
+                       join=True, start_method="spawn")
+    for r in range(world):
+        res = ast.literal_eval(str(np.load(tmp_path / f"x{r}.npy")[0]))
+        if fail_rank is None:
+            assert res["configured"] == (r, world)
+            assert res["peers"] == {p: p + 1 for p in range(world) if p != r}
+        else:
+            assert f"ranks [{fail_rank}]" in res["error"]
+            assert res["peers"] == {}  # nobody maps anything
