@@ -89,6 +89,7 @@ constexpr int kSegBars = 32;          // segment hand-off barriers (epilogue -> 
 enum TraceSlot {
     TR_START = 0, TR_XREADY, TR_FIRST_MMA, TR_QKV_DONE, TR_EPI_DONE, TR_XQ_DONE, TR_GATES_DONE,
     TR_UNIT0 = 7,  /* units 0, 1: claimed, (unused), done */
+    TR_GRID_WAIT = 13, /* the preceding grid has completed (griddepcontrol.wait returned) */
     TR_UNIT_HAND = 15, /* units 0, 1: o handed off */
     TR_PUB0 = 25, /* publisher: release of segment k issued and done, k < 7 */
     TR_O_WAIT0 = 19, TR_O_READY0, TR_O_READY_LAST, TR_END, TR_LAST_REDUCE_START, TR_LAST_REDUCE_END,
@@ -321,14 +322,24 @@ __device__ __forceinline__ bool wait_rb(const FusedParams &P, int key, const Ctl
 
 // ---------------------------------------------------------------- activation planes
 
-// Smallest power of two s with amax / s <= 448 (s = 1 for amax == 0).
+// Smallest power of two s with amax / s <= 448 (s = 1 for amax == 0), from the exponent
+// bits of amax / 448: that exponent, or the next one when amax / 448 is not itself a power of
+// two.  Below the normal range the scale stays at 2^-126.
 __device__ __forceinline__ float pow2_scale(float amax)
 {
     if (!(amax > 0.f)) return 1.f;
-    int e;
-    const float m = frexpf(amax * (1.f / 448.f), &e);
-    return ldexpf(1.f, m == 0.5f ? e - 1 : e);
+    const uint32_t y = __float_as_uint(amax * (1.f / 448.f));
+    uint32_t e = y >> 23;
+    if (e == 0u) return __uint_as_float(1u << 23);
+    if (y & 0x7FFFFFu) ++e;
+    return __uint_as_float(e << 23);
 }
+
+// 1 / s for a power of two s in [2^-126, 2^126] (exact).
+__device__ __forceinline__ float pow2_inv(float s) { return __uint_as_float((254u - (__float_as_uint(s) >> 23)) << 23); }
+
+// 1 / (1 + e^z) (the hardware exponential and reciprocal: a few ulp; 0 once e^z overflows).
+__device__ __forceinline__ float inv_one_plus_exp(float z) { return __fdividef(1.f, 1.f + __expf(z)); }
 
 // Row of plane p of sequence b in an x tile (2 planes; group b / 8) and in an o tile (4
 // planes; group 2 (b / 8) + p / 2).
@@ -403,13 +414,14 @@ __device__ void quantize_x(const FusedParams &P, int gw, int ngw, int lane)
 {
     constexpr ActGeo G = act_geo(BP);
     const int items = P.B * P.nKBx;
+#pragma unroll 1
     for (int it = gw; it < items; it += ngw) {
         const int b = it / P.nKBx, kb = it % P.nKBx;
         const uint2 raw = *reinterpret_cast<const uint2 *>(P.x + (size_t)b * P.H + kb * 128 + lane * 4);
         const float v0 = bf16_bits_to_float(raw.x & 0xFFFFu), v1 = bf16_bits_to_float(raw.x >> 16);
         const float v2 = bf16_bits_to_float(raw.y & 0xFFFFu), v3 = bf16_bits_to_float(raw.y >> 16);
         const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
-        const float s = pow2_scale(amax), inv = 1.f / s;  // exact: s is a power of two
+        const float s = pow2_scale(amax), inv = pow2_inv(s);  // exact: s is a power of two
         uint32_t w[2];
         split_planes<2>(v0 * inv, v1 * inv, v2 * inv, v3 * inv, w);
 #pragma unroll
@@ -431,11 +443,13 @@ __device__ void gate_rows(const FusedParams &P, VS *vs, int vt)
     const int vw = vt >> 5, lane = vt & 31;
     const int rows = P.nh + P.r;
     const int kchunk = P.H / 8;  // multiple of 16
+#pragma unroll 1
     for (int it = blockIdx.x; it < rows; it += gridDim.x) {
         const uint16_t *wrow = it < P.nh ? P.wb + (size_t)it * P.H : P.wa_down + (size_t)(it - P.nh) * P.H;
         float acc[BP];
 #pragma unroll
         for (int b = 0; b < BP; ++b) acc[b] = 0.f;
+#pragma unroll 1
         for (int k0 = vw * kchunk + lane * 8; k0 < (vw + 1) * kchunk; k0 += 256) {
             const uint4 wr = ld_stream_v4(wrow + k0);
             const uint32_t wv[4] = {wr.x, wr.y, wr.z, wr.w};
@@ -486,13 +500,14 @@ __device__ void gate_rows(const FusedParams &P, VS *vs, int vt)
 // Gates of state unit u (sequence u % B, o K-block u / B) into slot `slot`: beta of its
 // heads and alpha = exp(-softplus(z)) = 1 / (1 + e^z), z = W_a_up[row] . t, of its rows,
 // computed by vector threads [t0, t0 + nt).  t and W_b x must be final (C_GATE acquired).
-template <int DK, class VS>
+template <int DK, int DV, class VS>
 __device__ void unit_gates(const FusedParams &P, VS *vs, int u, int slot, int vt, int t0, int nt)
 {
-    const int b = u % P.Bs, kb = u / P.Bs, hpu = 128 / P.dv, h0 = kb * hpu;
+    constexpr int hpu = 128 / DV;
+    const int b = u % P.Bs, kb = u / P.Bs, h0 = kb * hpu;
     const int me = vt - t0;
     if (me < 0 || me >= nt) return;
-    if (me < hpu) vs->beta[slot][me] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + me)));
+    if (me < hpu) vs->beta[slot][me] = inv_one_plus_exp(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + me));
     const float *t = P.t + (size_t)b * P.r;
     for (int i = me; i < hpu * DK; i += nt) {
         const uint16_t *wr = P.wa_up + ((size_t)h0 * DK + i) * P.r;
@@ -518,17 +533,18 @@ __device__ void unit_gates(const FusedParams &P, VS *vs, int u, int slot, int vt
                 }
             }
         }
-        vs->a[slot][i] = 1.f / (1.f + expf(z));
+        vs->a[slot][i] = inv_one_plus_exp(z);
     }
 }
 
 // Gates of this CTA's first two units (u1 < 0: none) into slots 0 and 1, by all 256 vector
 // threads with every load issued in one batch: t of the two sequences into shared memory,
 // beta, and one W_a_up row per thread and unit.  t and W_b x must be final.
-template <int DK, class VS>
+template <int DK, int DV, class VS>
 __device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt)
 {
-    const int hpu = 128 / P.dv, rows = hpu * DK, r4 = P.r / 4;
+    constexpr int hpu = 128 / DV, rows = hpu * DK;
+    const int r4 = P.r / 4;
     const int us[2] = {u0, u1};
     float *ts = &vs->red_w[0][0];  // [2][r] (r <= 256)
     if (vt < 2 * r4) {
@@ -540,7 +556,7 @@ __device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt
         const int j = (vt - 128) / hpu, hh = (vt - 128) % hpu;
         if (us[j] >= 0) {
             const int b = us[j] % P.Bs, h = (us[j] / P.Bs) * hpu + hh;
-            vs->beta[j][hh] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)b * P.nh + h)));
+            vs->beta[j][hh] = inv_one_plus_exp(-__ldcg(P.bpre + (size_t)b * P.nh + h));
         }
     }
     for (int idx0 = 0; idx0 < 2 * rows; idx0 += 256) {
@@ -569,7 +585,7 @@ __device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt
                 }
             }
         }
-        if (has) vs->a[j][i] = 1.f / (1.f + expf(z));
+        if (has) vs->a[j][i] = inv_one_plus_exp(z);
     }
     named_bar(2, 256);
 }
@@ -577,10 +593,11 @@ __device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt
 // Gates of every token of a multi-token unit (sequence bs, o K-block kb): alpha into a[t],
 // beta into beta[t].  Each thread loads one W_a_up row once and dots it with the T rows of t
 // (staged in shared memory).  t and W_b x must be final.
-template <int DK, class VS>
+template <int DK, int DV, class VS>
 __device__ void token_gates(const FusedParams &P, VS *vs, int bs, int kb, int vt)
 {
-    const int T = P.T, hpu = 128 / P.dv, rows = hpu * DK, h0 = kb * hpu, r4 = P.r / 4;
+    constexpr int hpu = 128 / DV, rows = hpu * DK;
+    const int T = P.T, h0 = kb * hpu, r4 = P.r / 4;
     float *ts = &vs->red_w[0][0];  // [T][r], T * r <= 2048 (red_w and red_p)
     for (int idx = vt; idx < T * r4; idx += 256) {
         const int t = idx / r4, c4 = idx % r4;
@@ -589,7 +606,7 @@ __device__ void token_gates(const FusedParams &P, VS *vs, int bs, int kb, int vt
     }
     for (int idx = vt; idx < T * hpu; idx += 256) {
         const int t = idx / hpu, hh = idx % hpu;
-        vs->beta[t][hh] = 1.f / (1.f + expf(-__ldcg(P.bpre + (size_t)(bs * T + t) * P.nh + h0 + hh)));
+        vs->beta[t][hh] = inv_one_plus_exp(-__ldcg(P.bpre + (size_t)(bs * T + t) * P.nh + h0 + hh));
     }
     for (int i0 = 0; i0 < rows; i0 += 256) {
         const int i = i0 + vt;
@@ -628,7 +645,7 @@ __device__ void token_gates(const FusedParams &P, VS *vs, int bs, int kb, int vt
         if (has)
 #pragma unroll
             for (int t = 0; t < kMaxT; ++t)
-                if (t < T) vs->a[t][i] = 1.f / (1.f + expf(z[t]));
+                if (t < T) vs->a[t][i] = inv_one_plus_exp(z[t]);
     }
     named_bar(2, 256);
 }
@@ -638,14 +655,15 @@ __device__ void token_gates(const FusedParams &P, VS *vs, int bs, int kb, int vt
 // its gates are in slot nu & 1 and, while a few threads wait for the unit's q/k/v, the others
 // compute the gates of this CTA's next unit (next_u >= 0) into the other slot; with several
 // tokens every token's gates are computed here.
-template <int BP, int DK, bool MT, class VS>
+template <int BP, int DK, int DV, bool MT, class VS>
 __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, int next_u, int vt, int nu)
 {
     constexpr ActGeo G = act_geo(BP);
     const int T = MT ? P.T : 1, bs = u % P.Bs, kb = u / P.Bs, slot = nu & 1;
     constexpr int RPW = DK / 8;  // rows per warp
     const int vw = vt >> 5, lane = vt & 31;
-    const int dv = P.dv, hpu = 128 / dv, h0 = kb * hpu;
+    constexpr int dv = DV, hpu = 128 / DV;
+    const int h0 = kb * hpu;
     const int vc = lane * 4, hh = vc / dv, cc = vc % dv, h = h0 + hh;
     const int Dk = P.nh * DK, Dv = P.nh * dv;
     float *S = P.state + (((size_t)bs * P.nh + h) * DK) * dv + cc;
@@ -659,6 +677,14 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
     if (vt == 0) vs->fail = 0;
     named_bar(2, 256);
     if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu);
+    if (nu == 0) {
+        // first unit, its state loads in flight: every CTA's gate rows (t and W_b x) final,
+        // then this unit's and the next unit's gates (with several tokens: per unit, below)
+        if (vt == 0 && !wait_count(P.ctr + C_GATE, P.t_gate, c, 10)) vs->fail = 1;
+        named_bar(2, 256);
+        if (vs->fail) return false;
+        if (!MT) first_gates<DK, DV>(P, vs, u, next_u, vt);
+    }
     // then the heads' q, k, v: wait for every segment of their row groups (one thread per
     // counter, so the round trips overlap), add the partials
     {
@@ -669,17 +695,17 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
                                     : (vt < 2 * nq ? P.nRGq + glo + (vt - nq) : 2 * P.nRGq + vlo + (vt - 2 * nq));
             if (!wait_rb(P, key, c, 11)) vs->fail = 1;
         }
-        if (!MT && next_u >= 0 && nu >= 1) unit_gates<DK>(P, vs, next_u, slot ^ 1, vt, 32, 224);
+        if (!MT && next_u >= 0 && nu >= 1) unit_gates<DK, DV>(P, vs, next_u, slot ^ 1, vt, 32, 224);
     }
     named_bar(2, 256);
     if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu + 1);
     if (vs->fail) return false;
     if (MT) {
-        token_gates<DK>(P, vs, bs, kb, vt);
+        token_gates<DK, DV>(P, vs, bs, kb, vt);
 #pragma unroll
         for (int r = 0; r < RPW; ++r) s[r] = ld_stream_f4(S + (size_t)(vw * RPW + r) * dv);
     }
-    const int nqk = hpu * DK, per = 2 * nqk + 128;
+    constexpr int nqk = hpu * DK, per = 2 * nqk + 128;
     {
         // items (token t, i): q and k rows of the unit's heads, then its 128 v columns; a
         // thread's items are loaded together (one memory round trip), then summed in slot order
@@ -734,7 +760,7 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
         ss = warp_sum(ss);
         kq = warp_sum(kq);
         if (lane == 0) {
-            const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+            const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
             vs->inv[t][hd] = inv;
             vs->kq[t][hd] = kq * inv;
         }
@@ -781,7 +807,7 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
             const int row = bs * T + t;
             const float4 o4 = *reinterpret_cast<const float4 *>(&vs->o[vc]);
             const float amax = warp_max(fmaxf(fmaxf(fabsf(o4.x), fabsf(o4.y)), fmaxf(fabsf(o4.z), fabsf(o4.w))));
-            const float sc = pow2_scale(amax), inv = 1.f / sc;
+            const float sc = pow2_scale(amax), inv = pow2_inv(sc);
             uint32_t wq[4];
             split_planes<4>(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv, wq);
 #pragma unroll
@@ -845,7 +871,7 @@ __device__ void prefetch_unit_state(const FusedParams &P, int u)
         bulk_prefetch_l2_hint(p + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
 }
 
-template <int BP, int DK, bool MT, class VS>
+template <int BP, int DK, int DV, bool MT, class VS>
 __device__ void vector_role(const FusedParams &P, VS *vs, const Ctl &c)
 {
     constexpr ActGeo G = act_geo(BP);
@@ -859,13 +885,6 @@ __device__ void vector_role(const FusedParams &P, VS *vs, const Ctl &c)
     // ...: the same units every step, so the next unit's gates are computed while the
     // current one waits for its q/k/v.
     const int units = P.Bs * P.nKBo;
-    if ((int)blockIdx.x < units) {
-        if (vt == 0) vs->ok = wait_count(P.ctr + C_GATE, P.t_gate, c, 10);  // t and W_b x final
-        named_bar(2, 256);
-        if (!vs->ok) return;
-        const int u1 = (int)(blockIdx.x + gridDim.x);
-        if (!MT) first_gates<DK>(P, vs, blockIdx.x, u1 < units ? u1 : -1, vt);  // else per unit
-    }
     for (int nu = 0, u = blockIdx.x; u < units; ++nu, u += gridDim.x) {
         if (vt == 0) vs->unit = should_stop(c) ? 1 : 0;
         named_bar(2, 256);
@@ -873,7 +892,7 @@ __device__ void vector_role(const FusedParams &P, VS *vs, const Ctl &c)
         if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu);
         const int next = u + (int)gridDim.x < units ? u + (int)gridDim.x : -1;
         if (vt == 0 && next >= 0) prefetch_unit_state(P, next);  // its state streams in meanwhile
-        if (!state_unit<BP, DK, MT>(P, vs, c, u, next, vt, nu)) return;
+        if (!state_unit<BP, DK, DV, MT>(P, vs, c, u, next, vt, nu)) return;
         if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
     }
     // out = sum of the W_o partials (both plane pairs): items of 32 output rows.  With tensor
@@ -1129,23 +1148,35 @@ struct EpiGeo {
     static_assert(NW % 64 == 0, "a slot's columns come in 64-column loads");
 };
 
-// One tile into the running sums of warp quarter q.  Thread t owns sequence (first of the
-// group) + t/4 and KPS columns; both of its planes arrive in the same load and are added
-// before the scale.
+// The activation scales thread t of warp quarter q needs from a stage (one per slot): read
+// before the stage is handed back, so that its refill does not wait for the TMEM reads.
 template <int GR, int N, bool O>
-__device__ __forceinline__ void epi_accumulate(uint32_t tq, int q, int t, const uint8_t *as, int RS, float fw0,
-                                               float fw1, float (&acc)[64])
+__device__ __forceinline__ void epi_scales(int q, int t, const uint8_t *as, int RS, float (&sa)[4])
 {
     using E = EpiGeo<GR, N>;
 #pragma unroll
     for (int gi = 0; gi < E::GPW; ++gi) {
-        const int v = q + 4 * gi, g = v % GR, part = v / GR;
+        const int v = q + 4 * gi, g = v % GR;
+        const int b = (O ? 8 * (g / 2) : 8 * g) + (t >> 2);
+        sa[gi] = v < E::SL ? staged_scale(as, RS, b) : 0.f;
+    }
+}
+
+// One tile into the running sums of warp quarter q.  Thread t owns sequence (first of the
+// group) + t/4 and KPS columns; both of its planes arrive in the same load and are added
+// before the scale.
+template <int GR, int N, bool O>
+__device__ __forceinline__ void epi_accumulate(uint32_t tq, int q, int t, const float (&sa)[4], float fw0, float fw1,
+                                               float (&acc)[64])
+{
+    using E = EpiGeo<GR, N>;
+#pragma unroll
+    for (int gi = 0; gi < E::GPW; ++gi) {
+        const int v = q + 4 * gi, part = v / GR;
         if (v < E::SL) {
             const int h = v / 8;
             const uint32_t lofs = (uint32_t)(16 * ((v % 8) / 4));
-            const int b = (O ? 8 * (g / 2) : 8 * g) + (t >> 2);
-            const float sa = staged_scale(as, RS, b);
-            const float f0 = fw0 * sa, f1 = fw1 * sa;
+            const float f0 = fw0 * sa[gi], f1 = fw1 * sa[gi];
             const int col0 = GR < 4 ? part * E::NW : 0;
 #pragma unroll
             for (int c8 = 0; c8 < E::NW / 64; ++c8) {
@@ -1235,15 +1266,17 @@ __device__ void epilogue_role(const FusedParams &P, const Ring &R, const TileEnt
         if (!dead && !warp_wait_bar(&R.mmad[s], (uint32_t)(i / R.S) & 1u, c, 8)) dead = true;
         if (!dead) {
             tc_fence_after();
+            float sa[4];
+            if (e.mat < 3) epi_scales<G.gx, G.nx, false>(q, t, R.a(s), G.rsx, sa);
+            else epi_scales<G.go, G.no, true>(q, t, R.a(s), G.rso, sa);
+            __syncwarp();
+            if (t == 0) mbar_arrive(&R.empty[s]);  // the MMA is done and the stage's scales are read
             const uint32_t tb = tq + (uint32_t)(buf * R.cols);
-            if (e.mat < 3) epi_accumulate<G.gx, G.nx, false>(tb, q, t, R.a(s), G.rsx, w0, w1, acc);
-            else epi_accumulate<G.go, G.no, true>(tb, q, t, R.a(s), G.rso, w0, w1, acc);
+            if (e.mat < 3) epi_accumulate<G.gx, G.nx, false>(tb, q, t, sa, w0, w1, acc);
+            else epi_accumulate<G.go, G.no, true>(tb, q, t, sa, w0, w1, acc);
             tc_fence_before();
             __syncwarp();
-            if (t == 0) {
-                mbar_arrive(&R.empty[s]);       // the stage's scales are read, the MMA is done
-                mbar_arrive(&R.accempty[buf]);  // the accumulator is read
-            }
+            if (t == 0) mbar_arrive(&R.accempty[buf]);  // the accumulator is read
             if (threadIdx.x == 128 && i < 32) KDA_TR(P, TR_TILE_EPI + i);
         }
         if (!(e.flags & kSegEnd)) continue;
@@ -1276,7 +1309,7 @@ __device__ void publisher(const FusedParams &P, const Ring &R, const TileEntry *
 
 // MT: several tokens per sequence (multi-token steps; a separate instantiation keeps the
 // single-token state unit's registers to itself)
-template <int BP, int DK, bool MT>
+template <int BP, int DK, int DV, bool MT>
 __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ FusedParams P)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -1353,6 +1386,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
     int pre = 0;
     if (warp == 0 && lane == 0) pre = preissue_weights<BP>(P, R, my, n);
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) KDA_TR(P, TR_GRID_WAIT);
     if (warp == 3 && lane == 0) prefetch_l2_slice(P.x, (size_t)P.B * P.H * 2);
 
     if (warp < 4) {  // single-lane roles: few registers
@@ -1372,7 +1406,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fused(const __grid_constant__ F
         if (threadIdx.x == 128) KDA_TR(P, TR_EPI_DONE);
     } else {  // state units: the registers the others gave up
         regs_inc<kRegsVector>();
-        vector_role<BP, DK, MT>(P, vs, c);
+        vector_role<BP, DK, DV, MT>(P, vs, c);
     }
     tc_fence_before();
     __syncthreads();
@@ -1455,25 +1489,36 @@ int row_group_keys(const Dims &d, const SchedGeo &g)
 
 size_t ctr_words(const Dims &d, int max_keys) { return C_FIXED + (size_t)d.Dv() / 128 + max_keys + 16; }
 
-template <int BP, int DK, bool MT>
-void *kernel_ptr() { return reinterpret_cast<void *>(&k_fused<BP, DK, MT>); }
+template <int BP, int DK, int DV, bool MT>
+void *kernel_ptr() { return reinterpret_cast<void *>(&k_fused<BP, DK, DV, MT>); }
 
 template <bool MT>
-void *pick_kernel_t(int BP, int DK)
+void *pick_kernel_t(int BP, int DK, int DV)
 {
-    switch (BP * 1000 + DK) {
-    case 8064: return kernel_ptr<8, 64, MT>();
-    case 8128: return kernel_ptr<8, 128, MT>();
-    case 16064: return kernel_ptr<16, 64, MT>();
-    case 16128: return kernel_ptr<16, 128, MT>();
-    case 32064: return kernel_ptr<32, 64, MT>();
-    case 32128: return kernel_ptr<32, 128, MT>();
-    case 64064: return kernel_ptr<64, 64, MT>();
-    case 64128: return kernel_ptr<64, 128, MT>();
+    switch (BP * 1000000 + DK * 1000 + DV) {
+    case 8064064: return kernel_ptr<8, 64, 64, MT>();
+    case 8064128: return kernel_ptr<8, 64, 128, MT>();
+    case 8128064: return kernel_ptr<8, 128, 64, MT>();
+    case 8128128: return kernel_ptr<8, 128, 128, MT>();
+    case 16064064: return kernel_ptr<16, 64, 64, MT>();
+    case 16064128: return kernel_ptr<16, 64, 128, MT>();
+    case 16128064: return kernel_ptr<16, 128, 64, MT>();
+    case 16128128: return kernel_ptr<16, 128, 128, MT>();
+    case 32064064: return kernel_ptr<32, 64, 64, MT>();
+    case 32064128: return kernel_ptr<32, 64, 128, MT>();
+    case 32128064: return kernel_ptr<32, 128, 64, MT>();
+    case 32128128: return kernel_ptr<32, 128, 128, MT>();
+    case 64064064: return kernel_ptr<64, 64, 64, MT>();
+    case 64064128: return kernel_ptr<64, 64, 128, MT>();
+    case 64128064: return kernel_ptr<64, 128, 64, MT>();
+    case 64128128: return kernel_ptr<64, 128, 128, MT>();
     default: return nullptr;
     }
 }
-void *pick_kernel(int BP, int DK, bool multi) { return multi ? pick_kernel_t<true>(BP, DK) : pick_kernel_t<false>(BP, DK); }
+void *pick_kernel(int BP, int DK, int DV, bool multi)
+{
+    return multi ? pick_kernel_t<true>(BP, DK, DV) : pick_kernel_t<false>(BP, DK, DV);
+}
 
 // Shared memory past the ring: barriers, the vector warps' area, the tile list (+ the 1 KB
 // alignment slack of the dynamic allocation).
@@ -1633,7 +1678,7 @@ cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const vo
     if (tokens < 1 || tokens > kMaxT || d.B % tokens) return cudaErrorNotSupported;
     const int BP = bp_for(d.B), cls = class_of(BP);
     const bool multi = tokens > 1;
-    void *kern = pick_kernel(BP, d.dk, multi);
+    void *kern = pick_kernel(BP, d.dk, d.dv, multi);
     if (!kern || cls >= fs.nclass) return cudaErrorNotSupported;
     const ActGeo g = act_geo(BP);
     const SchedGeo sg = fused_sched_geo(d, BP);

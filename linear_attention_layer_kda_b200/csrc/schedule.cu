@@ -11,13 +11,17 @@
 namespace kda {
 
 // Row groups of N = 256 weight rows while the epilogue's running sums allow it (fewer for
-// 32 and 64 sequences); runs of BP / 2 tiles (4 at most batch sizes) so that the partial sums
-// a run writes stay a small fraction of the weight bytes it streams.
+// 32 and 64 sequences).  Runs: short ones spread each row group over more SMs, so its last
+// partial sum lands sooner, but every run writes a partial sum (BP x N fp32) and adds one to
+// the consumers' reads.  Measured at hidden 4096 (32 heads of 128 x 128): 2 tiles for 8
+// sequences (31.9 us against 32.5 us with 4), 4 for 16 (41.6 us against 48.7 us with 8),
+// BP / 2 for 64 (250.7 us; 252.5 us with 4); 8 for 32 sequences lies between.
 SchedGeo fused_sched_geo(const Dims &dmax, int BP)
 {
     const ActGeo g = act_geo(BP);
     const int nkb = dmax.H / 128;
-    return SchedGeo{g.nx, g.no, std::max(1, std::min(nkb, std::max(4, BP / 2)))};
+    const int run = BP <= 8 ? 2 : (BP <= 16 ? 4 : (BP <= 32 ? 8 : BP / 2));
+    return SchedGeo{g.nx, g.no, std::max(1, std::min(nkb, run))};
 }
 
 // Tile order and segments.

@@ -59,7 +59,7 @@ SHAPES = [(4096, 32, 128, 128, 64), (6144, 48, 128, 128, 64), (256, 2, 64, 64, 6
           (1024, 16, 64, 128, 16)]
 
 
-@pytest.mark.parametrize("BP,want", [(8, (256, 256, 4)), (16, (256, 256, 8)), (32, (256, 128, 16)),
+@pytest.mark.parametrize("BP,want", [(8, (256, 256, 2)), (16, (256, 256, 4)), (32, (256, 128, 8)),
                                      (64, (128, 64, 32))])
 def test_sched_geo(lib, BP, want):
     assert sched_geo(lib, BP, 4096, 32, 128, 128, 64) == want
