@@ -181,12 +181,19 @@ KDA_API int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weight
  *                token t, read out after token t's update
  *   chunk        tokens per chunk: 16, 32 or 64 (0: 32)
  * Each head's state goes through the tokens `chunk` at a time: inside a chunk the tokens'
- * updates are one unit lower-triangular solve and dense products (decays taken in log space,
- * log alpha clamped at -30).  The projections run the five-kernel engine's GEMV kernels over
- * all rows.  batch and tokens are not limited by max_batch: the handle keeps a workspace of
- * the activations of batch * tokens rows, allocated (cudaMalloc; waiting for the device when
- * it grows) on the first call that needs it and freed by kda_decode_destroy.  Same errors
- * and stream ordering as kda_decode_step; KDA_ERR_OUT_OF_MEMORY if the workspace cannot grow.
+ * updates are one unit lower-triangular system and dense products (decays taken in log space,
+ * log alpha clamped at -30).  Two kernels: the first prepares every chunk of every head at
+ * once (normalised keys, decays, the inverse of the chunk's triangular matrix); the second
+ * walks the chunks in order, one CTA per sequence, head and slice of value columns.  The
+ * projections are bf16 tensor-core GEMMs (cuBLASLt): each FP8 weight, scaled by its block
+ * scale, is split into two bf16 parts (hi + lo, about 2^-17 of the weight), as are the fp32
+ * activations o and t, so the products keep fp32-level accuracy.  batch and tokens are not
+ * limited by max_batch: the handle keeps a workspace (the activations of batch * tokens rows,
+ * the bf16 splits of the weights, one record per chunk), allocated (cudaMalloc; waiting for the
+ * device when it grows) on the first call that needs it and freed by kda_decode_destroy.
+ * Same errors and stream ordering as kda_decode_step; KDA_ERR_OUT_OF_MEMORY if the workspace
+ * cannot grow; a record copy that does not land within the wait limit is reported as
+ * KDA_ERR_DEVICE_TIMEOUT by the next call or kda_decode_sync.
  */
 KDA_API int kda_prefill(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out, int batch,
                         int tokens, int chunk);

@@ -19,6 +19,8 @@ NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
     "-Xcompiler", "-fPIC", "-shared", "-Xcompiler", "-fvisibility=hidden",
 ]
+# the prefill's projection GEMMs (cuBLASLt, from the CUDA toolkit)
+LINK_FLAGS = ["-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 
 
 def sources():
@@ -38,7 +40,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc] + NVCC_FLAGS + ["-I" + INCLUDE, "-I" + CSRC] + sources() + ["-o", tmp]
+    cmd = [nvcc] + NVCC_FLAGS + ["-I" + INCLUDE, "-I" + CSRC] + sources() + LINK_FLAGS + ["-o", tmp]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "fused.cuh"
+#include "prefill_gemm.cuh"
 #include "status.h"
 
 struct kda_handle_s {
@@ -25,6 +26,7 @@ struct kda_handle_s {
     void *out_stage = nullptr;  // device staging of out for kda_decode_step_host
     kda::FusedState fused;
     void *pf_ws = nullptr;   // prefill workspace (activations of every row), grown on demand
+    kda::LtGemm *lt = nullptr;  // the prefill's GEMM library handle, created on first use
     size_t pf_bytes = 0;
     bool fatal = false;  // a kernel gave up draining its copies after an abort: never step again
     std::string last_error;
@@ -585,9 +587,16 @@ int kda_prefill(kda_handle h, const void *x, const kda_weights *w, float *state_
         return fail(h, KDA_ERR_INVALID_ARG, "state_inout overlaps x or out");
     rc = take_device_status(h);
     if (rc) return rc;
-    // workspace: the fp32 activations of every row
-    const size_t sizes[7] = {rows * Dk * 4, rows * Dk * 4, rows * Dk * 4, rows * Dv * 4, rows * Dv * 4,
-                             rows * (size_t)c.num_heads * 4, rows * (size_t)c.alpha_rank * 4};
+    if (!h->lt) {
+        const cudaError_t e0 = kda::lt_create(&h->lt);
+        if (e0 != cudaSuccess) return cuda_fail(h, e0, "GEMM library handle");
+    }
+    // workspace: the fp32 activations of every row, then the GEMMs' bf16 splits
+    const kda::Dims d = dims_of(c, (int)rows);
+    const size_t sizes[9] = {rows * Dk * 4, rows * Dk * 4, rows * Dk * 4, rows * Dv * 4, rows * Dv * 4,
+                             rows * (size_t)c.num_heads * 4, rows * (size_t)c.alpha_rank * 4,
+                             kda::prefill_gemm_ws_bytes(d),
+                             kda::chunk_ws_bytes(c.head_dk, c.num_heads, batch, tokens, chunk)};
     size_t need = 0;
     for (size_t sz : sizes) need += align_up(sz, 256);
     if (need > h->pf_bytes) {
@@ -607,10 +616,11 @@ int kda_prefill(kda_handle h, const void *x, const kda_weights *w, float *state_
         *dst[i] = reinterpret_cast<float *>(p);
         p += align_up(sizes[i], 256);
     }
-    const kda::Dims d = dims_of(c, (int)rows);
-    cudaError_t e = kda::simple_projections(d, *w, x, s, h->stream);
-    if (e == cudaSuccess) e = kda::chunk_state(d, batch, tokens, chunk, s, state_inout, h->stream);
-    if (e == cudaSuccess) e = kda::simple_out_projection(d, *w, s.o, out, c.out_dtype, h->stream);
+    void *gws = p, *cws = p + align_up(sizes[7], 256);
+    cudaError_t e = kda::prefill_projections(h->lt, d, *w, x, s, gws, h->stream);
+    if (e == cudaSuccess)
+        e = kda::chunk_state(d, batch, tokens, chunk, s, state_inout, cws, h->status, h->fused.timeout_ns, h->stream);
+    if (e == cudaSuccess) e = kda::prefill_out_projection(h->lt, d, *w, s.o, out, c.out_dtype, gws, h->stream);
     if (e != cudaSuccess) return cuda_fail(h, e, "prefill launch");
     return KDA_OK;
 }
@@ -683,6 +693,7 @@ int kda_decode_destroy(kda_handle h)
     if (cudaStreamSynchronize(h->stream) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     kda::fused_destroy(&h->fused);
     if (h->pf_ws && cudaFree(h->pf_ws) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    kda::lt_destroy(h->lt);
     for (int r = 0; r < h->fused.tp_world; ++r) {
         void *p = h->fused.tp_region[r];
         if (!p) continue;

@@ -48,11 +48,13 @@ cudaError_t simple_out_projection(const Dims &d, const kda_weights &w, const flo
                                   cudaStream_t st);
 
 // Chunked form of the recurrence for nseq sequences of T tokens (activations of row b*T + t in
-// s, as simple_projections leaves them): o of every token into s.o, the state advanced by T
-// tokens.  chunk: tokens per chunk (chunk_supported says which).
+// s, as the projections leave them): o of every token into s.o, the state advanced by T
+// tokens.  chunk: tokens per chunk (chunk_supported says which); ws: chunk_ws_bytes of device
+// workspace (the per-chunk records); a wait that exceeds timeout_ns is recorded in status.
 bool chunk_supported(int dk, int dv, int chunk);
-size_t chunk_smem_bytes(int dk, int dv, int chunk);
-cudaError_t chunk_state(const Dims &d, int nseq, int T, int chunk, const Scratch &s, float *state, cudaStream_t st);
+size_t chunk_ws_bytes(int dk, int nh, int nseq, int T, int chunk);
+cudaError_t chunk_state(const Dims &d, int nseq, int T, int chunk, const Scratch &s, float *state, void *ws,
+                        int *status, uint64_t timeout_ns, cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__
