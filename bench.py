@@ -512,12 +512,16 @@ def run_ours(args, shape, rank, world, local_rank):
     return 0
 
 
+FUSED_SOURCES = ("common.cuh", "fused.cu", "fused.cuh", "schedule.cu", "sm100.cuh")
+
+
 def kernel_rev() -> str:
-    """Hash of the CUDA sources: a stored ncu traffic figure is reported only for the kernel it measured."""
+    """Hash of the fused engine's sources: a stored ncu traffic figure is reported only for the
+    kernel it measured."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_attention_layer_kda_b200", "csrc")
-    for n in sorted(f for f in os.listdir(d) if f.endswith((".cu", ".cuh"))):  # the engines and the ABI
+    for n in FUSED_SOURCES:
         for line in open(os.path.join(d, n)):
             code = line.split("//", 1)[0].strip()  # comments and layout do not change the kernel
             if code:

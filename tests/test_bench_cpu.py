@@ -38,7 +38,11 @@ def test_kernel_revision_ignores_comments(tmp_path, monkeypatch):
     assert bench.kernel_rev() == rev
     with open(fake / "fused.cu", "a") as f:
         f.write("static int kda_extra_symbol_for_the_test = 1;\n")
-    assert bench.kernel_rev() != rev
+    rev2 = bench.kernel_rev()
+    assert rev2 != rev
+    with open(fake / "chunk.cu", "a") as f:  # the prefill kernels are not part of the fused engine
+        f.write("static int kda_other_engine_symbol = 1;\n")
+    assert bench.kernel_rev() == rev2
 
 
 def test_step_percentiles():
