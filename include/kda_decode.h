@@ -152,6 +152,19 @@ KDA_API int kda_decode_step_host(kda_handle h, const void *x_host, const kda_wei
                          void *out_host, int batch);
 
 /*
+ * The same step from host buffers, without waiting: for a loop that feeds steps from the
+ * host and reads every result.  x is copied in and out is copied back on two copy streams of
+ * the handle (created with two device staging slots on the first call), so the copies of one
+ * step overlap the neighbouring steps' kernels; the steps themselves stay in order on the
+ * handle's stream.  x_host and out_host should be page-locked (pageable memory makes the
+ * copies synchronous).  x_host may be reused, and out_host read, only after kda_decode_sync(h),
+ * which waits for all of the handle's streams.  Same arguments and errors as kda_decode_step_host, plus
+ * KDA_ERR_OUT_OF_MEMORY if the staging cannot be allocated.
+ */
+KDA_API int kda_decode_step_host_async(kda_handle h, const void *x_host, const kda_weights *w, float *state_inout,
+                                       void *out_host, int batch);
+
+/*
  * Several tokens per sequence in one call: `tokens` consecutive tokens of each of `batch`
  * sequences, as in the verify step of multi-token (speculative) decoding that the Kiln post
  * ("What did we measure that did not pay?") and the TileRT README (MTP) describe.
@@ -265,8 +278,9 @@ KDA_API int kda_decode_set_launch_overlap(kda_handle h, int on);
 KDA_API int kda_tp_configure(kda_handle h, int rank, int world, void *handle_out);
 KDA_API int kda_tp_set_peer(kda_handle h, int peer, const void *handle);
 
-/* Waits for the handle's stream; returns the device status of the steps since
- * the last check (KDA_OK or KDA_ERR_DEVICE_TIMEOUT) and clears it. */
+/* Waits for the handle's stream (and its copy streams, if kda_decode_step_host_async made them);
+ * returns the device status of the steps since the last check (KDA_OK or
+ * KDA_ERR_DEVICE_TIMEOUT) and clears it. */
 KDA_API int kda_decode_sync(kda_handle h);
 
 /* Frees the handle's scratch.  Waits for its stream first.  NULL is accepted. */

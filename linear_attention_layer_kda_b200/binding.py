@@ -35,7 +35,7 @@ EXPORTS = (
     "kda_status_string", "kda_decode_last_error", "kda_decode_abi_version", "kda_decode_debug_copy",
     "kda_decode_step_noalloc", "kda_decode_step_tokens", "kda_state_checkpoint", "kda_state_restore",
     "kda_decode_set_launch_overlap", "kda_decode_tokens_engine", "kda_prefill", "kda_tp_configure",
-    "kda_tp_set_peer",
+    "kda_tp_set_peer", "kda_decode_step_host_async",
 )
 KDA_TP_HANDLE_BYTES = 64
 KDA_NOALLOC_MAX_SCRATCH_BYTES = 1 << 20
@@ -102,6 +102,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kda_prefill": (I, [P, P, ctypes.POINTER(kda_weights), P, P, I, I, I]),
         "kda_tp_configure": (I, [P, I, I, P]),
         "kda_tp_set_peer": (I, [P, I, P]),
+        "kda_decode_step_host_async": (I, [P, P, ctypes.POINTER(kda_weights), P, P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -150,6 +151,11 @@ def kda_state_restore(h: int, host_src: int, state: int, seq0: int, nseq: int) -
 
 def kda_decode_step_host(h: int, x_host: int, w: kda_weights, state: int, out_host: int, batch: int) -> None:
     _check(load().kda_decode_step_host(h, x_host, ctypes.byref(w), state, out_host, batch), "kda_decode_step_host", h)
+
+
+def kda_decode_step_host_async(h: int, x_host: int, w: kda_weights, state: int, out_host: int, batch: int) -> None:
+    _check(load().kda_decode_step_host_async(h, x_host, ctypes.byref(w), state, out_host, batch),
+           "kda_decode_step_host_async", h)
 
 
 def kda_decode_set_launch_overlap(h: int, on: bool) -> None:
@@ -269,6 +275,13 @@ class KdaDecoder:
         b = x_host.shape[0] if batch is None else batch
         self._bind_stream()
         kda_decode_step_host(self.h, x_host.data_ptr(), weights, state.data_ptr(), out_host.data_ptr(), b)
+
+    def step_host_async(self, x_host, weights: kda_weights, state, out_host, batch: Optional[int] = None) -> None:
+        """Host-buffer step without waiting (copies on the handle's copy stream); out_host is
+        valid after sync()."""
+        b = x_host.shape[0] if batch is None else batch
+        self._bind_stream()
+        kda_decode_step_host_async(self.h, x_host.data_ptr(), weights, state.data_ptr(), out_host.data_ptr(), b)
 
     def step_tokens(self, x, weights: kda_weights, state, out, batch: int, tokens: int) -> None:
         """`tokens` tokens of each of `batch` sequences; x and out are [batch * tokens, H]."""

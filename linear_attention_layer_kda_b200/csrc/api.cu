@@ -24,6 +24,12 @@ struct kda_handle_s {
     int *status = nullptr;       // its device alias; kernels record KDA_ERR_DEVICE_TIMEOUT here
     void *x_stage = nullptr;    // device staging of x for kda_decode_step_host
     void *out_stage = nullptr;  // device staging of out for kda_decode_step_host
+    // kda_decode_step_host_async: two staging slots, copy streams in and out and their events
+    // (created on first use)
+    void *hx[2] = {}, *hout[2] = {};
+    cudaStream_t cstream = nullptr, ostream = nullptr;
+    cudaEvent_t ev_x[2] = {}, ev_k[2] = {}, ev_o[2] = {};
+    int hslot = 0;
     kda::FusedState fused;
     void *pf_ws = nullptr;   // prefill workspace (activations of every row), grown on demand
     kda::LtGemm *lt = nullptr;  // the prefill's GEMM library handle, created on first use
@@ -528,6 +534,67 @@ int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w,
     return take_device_status(h);
 }
 
+static int host_async_setup(kda_handle h)
+{
+    if (h->ostream) return KDA_OK;
+    const size_t B = (size_t)h->cfg.max_batch, H = (size_t)h->cfg.hidden;
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+        e = cudaMalloc(&h->hx[i], B * H * 2);
+        if (e == cudaSuccess) e = cudaMalloc(&h->hout[i], B * H * 4);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_x[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_k[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_o[i], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cstream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->ostream, cudaStreamNonBlocking);
+    // the slots start free: their "step done" and "out copied" events complete at once
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+        e = cudaEventRecord(h->ev_k[i], h->cstream);
+        if (e == cudaSuccess) e = cudaEventRecord(h->ev_o[i], h->ostream);
+    }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(h, KDA_ERR_OUT_OF_MEMORY, "host-step staging allocation failed");
+    }
+    return KDA_OK;
+}
+
+int kda_decode_step_host_async(kda_handle h, const void *x_host, const kda_weights *w, float *state_inout,
+                               void *out_host, int batch)
+{
+    if (!h) return KDA_ERR_INVALID_ARG;
+    if (!x_host || !out_host) return fail(h, KDA_ERR_INVALID_ARG, "null host buffer");
+    int rc = check_usable(h);
+    if (rc) return rc;
+    rc = host_async_setup(h);
+    if (rc) return rc;
+    const int s = h->hslot;
+    rc = check_step(h, h->hx[s], w, state_inout, h->hout[s], batch);
+    if (rc) return rc;
+    rc = take_device_status(h);
+    if (rc) return rc;
+    const size_t nx = (size_t)batch * h->cfg.hidden * 2;
+    const size_t no = (size_t)batch * h->cfg.hidden * (h->cfg.out_dtype == KDA_OUT_BF16 ? 2 : 4);
+    // in: once the step that last used slot s has read its x; the step: once x is in and the
+    // slot's previous out has been copied back; out: once the step is done
+    cudaError_t e = cudaStreamWaitEvent(h->cstream, h->ev_k[s], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(h->hx[s], x_host, nx, cudaMemcpyHostToDevice, h->cstream);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_x[s], h->cstream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->stream, h->ev_x[s], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->stream, h->ev_o[s], 0);
+    if (e != cudaSuccess) return cuda_fail(h, e, "copying x to the device");
+    rc = enqueue_step(h, h->hx[s], w, state_inout, h->hout[s], batch);
+    if (rc) return rc;
+    e = cudaEventRecord(h->ev_k[s], h->stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->ostream, h->ev_k[s], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(out_host, h->hout[s], no, cudaMemcpyDeviceToHost, h->ostream);
+    if (e == cudaSuccess) e = cudaEventRecord(h->ev_o[s], h->ostream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "copying out to the host");
+    h->hslot = s ^ 1;
+    return KDA_OK;
+}
+
 int kda_decode_step_tokens(kda_handle h, const void *x, const kda_weights *w, float *state_inout, void *out,
                            int batch, int tokens)
 {
@@ -655,6 +722,8 @@ int kda_decode_sync(kda_handle h)
 {
     if (!h) return KDA_ERR_INVALID_ARG;
     cudaError_t e = cudaStreamSynchronize(h->stream);
+    if (e == cudaSuccess && h->cstream) e = cudaStreamSynchronize(h->cstream);
+    if (e == cudaSuccess && h->ostream) e = cudaStreamSynchronize(h->ostream);
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
     const int st = take_device_status(h);
     return st ? st : check_usable(h);
@@ -691,6 +760,18 @@ int kda_decode_destroy(kda_handle h)
     if (!h) return KDA_OK;
     int rc = KDA_OK;
     if (cudaStreamSynchronize(h->stream) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+    for (cudaStream_t cs : {h->cstream, h->ostream}) {
+        if (!cs) continue;
+        if (cudaStreamSynchronize(cs) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
+        (void)cudaStreamDestroy(cs);
+    }
+    for (int i = 0; i < 2; ++i) {
+        if (h->ev_x[i]) (void)cudaEventDestroy(h->ev_x[i]);
+        if (h->ev_k[i]) (void)cudaEventDestroy(h->ev_k[i]);
+        if (h->ev_o[i]) (void)cudaEventDestroy(h->ev_o[i]);
+        if (h->hx[i]) (void)cudaFree(h->hx[i]);
+        if (h->hout[i]) (void)cudaFree(h->hout[i]);
+    }
     kda::fused_destroy(&h->fused);
     if (h->pf_ws && cudaFree(h->pf_ws) != cudaSuccess) { (void)cudaGetLastError(); rc = KDA_ERR_CUDA; }
     kda::lt_destroy(h->lt);

@@ -111,6 +111,36 @@ def test_replays_are_bitwise_identical():
     dec.close()
 
 
+def test_pipelined_host_steps_match_device_steps():
+    """kda_decode_step_host_async: six steps fed from pinned host buffers without waiting, each
+    out copied to its own host buffer, give the device steps' bits (out of every step, state)."""
+    import torch
+    from linear_attention_layer_kda_b200 import tensors
+    shape = I.CONFIGS[1].replace(steps=6)
+    inp = I.generate(shape)
+    B, H = shape.batch, shape.hidden
+    w = tensors.weights_struct(tensors.to_device_weights(inp))
+    dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, B)
+    try:
+        s_dev, s_host = tensors.state_tensor(inp.state0), tensors.state_tensor(inp.state0)
+        ref = []
+        for t in range(shape.steps):
+            out = torch.empty(B, H, device="cuda")
+            dec.step(tensors.bf16_tensor(inp.x[t]), w, s_dev, out)
+            ref.append(out)
+        dec.sync()
+        xh = [torch.from_numpy(inp.x[t].view(np.int16)).view(torch.bfloat16).pin_memory() for t in range(shape.steps)]
+        oh = [torch.full((B, H), float("nan")).pin_memory() for _ in range(shape.steps)]
+        for t in range(shape.steps):
+            dec.step_host_async(xh[t], w, s_host, oh[t])
+        dec.sync()
+        for t in range(shape.steps):
+            assert torch.equal(oh[t], ref[t].cpu()), f"step {t}"
+        assert torch.equal(s_host, s_dev)
+    finally:
+        dec.close()
+
+
 def test_host_buffer_entry_point_matches_device_entry_point():
     import torch
     from linear_attention_layer_kda_b200 import tensors

@@ -94,6 +94,36 @@ def test_chunk_sizes_agree():
         assert maxrel(o, res[0][0]) <= 1e-4 and maxrel(s, res[0][1]) <= 1e-4
 
 
+def test_prefill_bf16_out_and_growing_workspace():
+    """bf16 out (the output GEMMs sum in fp32, then one rounding) and one handle whose workspace
+    grows between calls: a short prompt, then a longer one continuing the same state."""
+    import torch
+    from linear_attention_layer_kda_b200 import tensors
+    shape = RAGGED
+    T1, T2 = 40, 200
+    inp = I.generate(shape.replace(steps=T1 + T2))
+    B, H = shape.batch, shape.hidden
+    w = tensors.weights_struct(tensors.to_device_weights(inp))
+    dec = binding.KdaDecoder(H, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank, B,
+                             out_dtype=binding.KDA_OUT_BF16)
+    ref_out, ref_state = _oracle(inp, shape, T1 + T2)
+    try:
+        st = tensors.state_tensor(inp.state0)
+        got = []
+        for t0, T in ((0, T1), (T1, T2)):
+            xs = tensors.bf16_tensor(np.stack([inp.x[t] for t in range(t0, t0 + T)], axis=1).reshape(B * T, H))
+            out = torch.full((B * T, H), float("nan"), device="cuda", dtype=torch.bfloat16)
+            dec.prefill(xs, w, st, out, B, T, 32)
+            dec.sync()
+            got.append(out.view(B, T, H).double().cpu().numpy())
+        got_out = np.concatenate(got, axis=1)
+        worst = max(maxrel(got_out[:, t], ref_out[:, t]) for t in range(T1 + T2))
+        assert worst <= OUT_TOL + 2.0 ** -9, f"out error {worst:.3e}"
+        assert maxrel(st.double().cpu().numpy(), ref_state) <= STATE_TOL
+    finally:
+        dec.close()
+
+
 def test_prefill_argument_errors():
     import ctypes
     s = I.CONFIGS[0]
