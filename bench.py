@@ -298,9 +298,10 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
-def job_steps_per_s(ms_per_step_slowest: float, world: int) -> float:
-    """Whole-job decode steps/s: every rank advances its own batch once per step."""
-    return world * 1000.0 / ms_per_step_slowest
+def job_steps_per_s(ms_per_step_slowest: float, world: int, tp: bool = False) -> float:
+    """Whole-job decode steps/s: every rank advances its own batch once per step (data
+    parallel), or all ranks advance one batch together (tensor parallel by heads)."""
+    return (1 if tp else world) * 1000.0 / ms_per_step_slowest
 
 
 def step_percentiles(step_ms):
@@ -328,7 +329,13 @@ def run_ours(args, shape, rank, world, local_rank):
     TK = args.tokens if args.prefill <= 0 else args.prefill
     if TK > 1:
         shape = shape.replace(steps=max(shape.steps, TK))
-    inp = rank_inputs(shape, rank, world)
+    full_shape = shape
+    if args.tp:  # this rank's heads: their weights and state, x and W_a_down whole
+        from linear_attention_layer_kda_b200 import tp
+        inp = tp.shard_inputs(I.generate(shape.replace(steps=max(1, shape.steps))), rank, world)
+        shape = inp.shape
+    else:
+        inp = rank_inputs(shape, rank, world)
     T = len(inp.x)  # fresh x per step for multi-step workloads
     set_bytes = ideal_bytes(shape, B, tokens=TK)
     R = rotation_sets(shape, l2)
@@ -344,6 +351,9 @@ def run_ours(args, shape, rank, world, local_rank):
     prefill = args.prefill > 0
     dec = binding.KdaDecoder(shape.hidden, shape.num_heads, shape.head_dk, shape.head_dv, shape.alpha_rank,
                              B if prefill else B * TK, engine=args.engine)
+    if args.tp:  # the out sum over ranks inside the fused kernel, over peer memory
+        from linear_attention_layer_kda_b200 import tp
+        tp.exchange_handles(dec, rank, world)
     if prefill:
         # this library's kernels per call (weight and activation splits, the chunk preparation and
         # scan) and the cuBLASLt GEMMs of the projections, beside them
@@ -413,7 +423,7 @@ def run_ours(args, shape, rank, world, local_rank):
 
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_per_step = ms_total / args.steps
-    value = job_steps_per_s(ms_per_step, world)
+    value = job_steps_per_s(ms_per_step, world, args.tp)
     med, p10, p90 = step_percentiles(step_ms)
 
     # end to end through the host-buffer entry point: H2D x, step, D2H out, sync, every step,
@@ -442,10 +452,10 @@ def run_ours(args, shape, rank, world, local_rank):
         for i in range(n_e2e):
             dec.step_host(xh[i % T], ws[i % R], states[i % R], oh)
         dtb = max_over_ranks(time.perf_counter() - t0, world, dev)
-        e2e = {"value": job_steps_per_s(1000.0 * dt / n_e2e, world), "unit": "steps/s",
+        e2e = {"value": job_steps_per_s(1000.0 * dt / n_e2e, world, args.tp), "unit": "steps/s",
                "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(oh.numel() * 4),
                "steps": n_e2e, "call": "kda_decode_step_host_async every step, one kda_decode_sync at the end",
-               "blocking": {"value": job_steps_per_s(1000.0 * dtb / n_e2e, world), "unit": "steps/s",
+               "blocking": {"value": job_steps_per_s(1000.0 * dtb / n_e2e, world, args.tp), "unit": "steps/s",
                             "call": "kda_decode_step_host (waits for its result) every step"}}
 
     cpu = None
@@ -472,7 +482,7 @@ def run_ours(args, shape, rank, world, local_rank):
     ib = ideal_bytes(shape, B, tokens=TK)
     achieved = ib / (ms_per_step * 1e-3) / 1e9
     traffic = None
-    tfile = os.path.join(ROOT, "profiles", f"traffic_{shape.name}.json")
+    tfile = os.path.join(ROOT, "profiles", f"traffic_{shape.name}.json")  # (a head shard has its own name)
     if os.path.exists(tfile):
         try:
             tj = json.load(open(tfile))
@@ -503,9 +513,14 @@ def run_ours(args, shape, rank, world, local_rank):
                             "work is not counted"}
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if args.tp else "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(shape, world, R), **({"tokens_per_step": TK} if TK > 1 else {})),
+        "config": dict(workload_config(full_shape, 1 if args.tp else world, R),
+                       **({"tokens_per_step": TK} if TK > 1 else {}),
+                       **({"parallelism": f"tp{world} (heads split over the ranks, {shape.num_heads} per rank; the out "
+                                          f"all-reduce inside the fused kernel over peer memory)"}
+                          if args.tp else {})),
         "tokens_per_s": value * B * TK,
         "step_us": {"median": med * 1e3, "p10": p10 * 1e3, "p90": p90 * 1e3,
                     "note": "second pass, an event after every step on the launching stream (rank 0); "
@@ -570,6 +585,9 @@ def parse_args(argv=None):
     ap.add_argument("--clock-window", type=float, default=0.5,
                     help="seconds of untimed steps before the timed region, so clocks settle under load")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the host-buffer end-to-end loop")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor parallel by heads over the N ranks (the out all-reduce inside the kernel); "
+                         "default: data parallel over sequences")
     ap.add_argument("--tokens", type=int, default=1,
                     help="tokens per sequence in one step (multi-token verify through kda_decode_step_tokens)")
     ap.add_argument("--prefill", type=int, default=0, help="time kda_prefill of this many tokens per sequence")

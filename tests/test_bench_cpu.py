@@ -23,6 +23,7 @@ def test_algorithmic_bytes_by_hand_at_batch_8():
 def test_job_rate_counts_every_rank():
     assert bench.job_steps_per_s(0.05, 1) == 20000.0
     assert bench.job_steps_per_s(0.05, 8) == 160000.0
+    assert bench.job_steps_per_s(0.05, 8, tp=True) == 20000.0  # the ranks advance one batch together
 
 
 def test_kernel_revision_ignores_comments(tmp_path, monkeypatch):
