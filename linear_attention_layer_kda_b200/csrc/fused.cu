@@ -774,15 +774,24 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
         const float *kt = vs->k[t], *qt = vs->q[t];
         // S~ = diag(alpha) S; partial w = S~^T k^, p = S~^T q over this warp's rows
         float4 pw = make_float4(0.f, 0.f, 0.f, 0.f), pp = pw;
+        const int i0 = hh * DK + vw * RPW;  // this warp's rows, four at a time (16-byte loads)
 #pragma unroll
-        for (int r = 0; r < RPW; ++r) {
-            const int i = hh * DK + vw * RPW + r;
-            const float a = al[i], kk = kt[i], qq = qt[i];
-            s[r].x *= a; s[r].y *= a; s[r].z *= a; s[r].w *= a;
-            pw.x = fmaf(kk, s[r].x, pw.x); pw.y = fmaf(kk, s[r].y, pw.y);
-            pw.z = fmaf(kk, s[r].z, pw.z); pw.w = fmaf(kk, s[r].w, pw.w);
-            pp.x = fmaf(qq, s[r].x, pp.x); pp.y = fmaf(qq, s[r].y, pp.y);
-            pp.z = fmaf(qq, s[r].z, pp.z); pp.w = fmaf(qq, s[r].w, pp.w);
+        for (int r4 = 0; r4 < RPW; r4 += 4) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(al + i0 + r4);
+            const float4 k4 = *reinterpret_cast<const float4 *>(kt + i0 + r4);
+            const float4 q4 = *reinterpret_cast<const float4 *>(qt + i0 + r4);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float4 &sr = s[r4 + j];
+                const float a = av[j], kk = kv[j], qq = qv[j];
+                sr.x *= a; sr.y *= a; sr.z *= a; sr.w *= a;
+                pw.x = fmaf(kk, sr.x, pw.x); pw.y = fmaf(kk, sr.y, pw.y);
+                pw.z = fmaf(kk, sr.z, pw.z); pw.w = fmaf(kk, sr.w, pw.w);
+                pp.x = fmaf(qq, sr.x, pp.x); pp.y = fmaf(qq, sr.y, pp.y);
+                pp.z = fmaf(qq, sr.z, pp.z); pp.w = fmaf(qq, sr.w, pp.w);
+            }
         }
         *reinterpret_cast<float4 *>(&vs->red_w[vw][vc]) = pw;
         *reinterpret_cast<float4 *>(&vs->red_p[vw][vc]) = pp;
@@ -821,10 +830,15 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
         // S' = S~ + k^ u^T (kept in registers for the next token)
         const float4 u4 = *reinterpret_cast<const float4 *>(&vs->u[vc]);
 #pragma unroll
-        for (int r = 0; r < RPW; ++r) {
-            const float kk = kt[hh * DK + vw * RPW + r];
-            s[r].x = fmaf(kk, u4.x, s[r].x); s[r].y = fmaf(kk, u4.y, s[r].y);
-            s[r].z = fmaf(kk, u4.z, s[r].z); s[r].w = fmaf(kk, u4.w, s[r].w);
+        for (int r4 = 0; r4 < RPW; r4 += 4) {
+            const float4 k4 = *reinterpret_cast<const float4 *>(kt + i0 + r4);
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float4 &sr = s[r4 + j];
+                sr.x = fmaf(kv[j], u4.x, sr.x); sr.y = fmaf(kv[j], u4.y, sr.y);
+                sr.z = fmaf(kv[j], u4.z, sr.z); sr.w = fmaf(kv[j], u4.w, sr.w);
+            }
         }
         if (t + 1 < T) named_bar(2, 256);  // u, o and the reductions are reused by the next token
     }
