@@ -213,8 +213,7 @@ __global__ void __launch_bounds__(kChunkThreads)
 template <int DK, int DV, int C, int NBUF>
 struct ScanSmem {
     using R = ChunkRec<DK, C>;
-    static constexpr int S = 0;
-    static constexpr int REC = (DK * DV + 31) / 32 * 32;
+    static constexpr int REC = (DK * DV + 31) / 32 * 32;  // S at offset 0
     static constexpr int RSTRIDE = (R::TOTAL + 31) / 32 * 32;
     static constexpr int UB = REC + NBUF * RSTRIDE;
     static constexpr int BARS = UB + C * DV;
@@ -263,7 +262,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     using L = ScanSmem<DK, DV, C, NBUF>;
     constexpr int JB = DV / 4, TB = kChunkThreads / JB, RD = DK / TB;
     static_assert(TB == C, "one token row per thread");
-    float *S = sm + L::S, *UB = sm + L::UB;
+    float *S = sm, *UB = sm + L::UB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
     __shared__ int stop;
     const int h = blockIdx.x, b = blockIdx.y, col0 = blockIdx.z * DV, tid = threadIdx.x;
