@@ -105,6 +105,8 @@ enum TraceSlot {
 //   off_oready+kb state units done for o K-block kb (B per step)
 //   off_rb+key    segments published for row group key (q, k, v, o row groups)
 constexpr int C_XQ = 0, C_GATE = 1, C_ABORT = 4, C_FIXED = 16;
+// Gate buffer: per state unit, alpha of its rows at [0, 256) and beta of its heads at kGateBeta.
+constexpr int kGateBeta = 256, kGateStride = 260;
 
 // Status words in mapped host memory: [0] status, [1] wait site, [2] set when a drain of
 // copies in flight gave up (the handle can no longer be trusted).
@@ -144,6 +146,7 @@ struct FusedParams {
     void *out;
     uint8_t *xq, *oq;  // x and o planes + scale rows
     float *part;
+    float *gbuf;  // single-token gates of every state unit [units][kGateStride]
     float *q, *k, *v, *bpre, *t;
     uint32_t *ctr;
     uint64_t *trace;  // null unless built with KDA_TRACE
@@ -497,51 +500,12 @@ __device__ void gate_rows(const FusedParams &P, VS *vs, int vt)
     }
 }
 
-// Gates of state unit u (sequence u % B, o K-block u / B) into slot `slot`: beta of its
-// heads and alpha = exp(-softplus(z)) = 1 / (1 + e^z), z = W_a_up[row] . t, of its rows,
-// computed by vector threads [t0, t0 + nt).  t and W_b x must be final (C_GATE acquired).
+// Gates of two units (u1 < 0: none) into their rows of the gate buffer (alpha of the unit's
+// rows at [0, hpu * dk), beta of its heads at kGateBeta), by all 256 vector threads with every
+// load issued in one batch: t of the two sequences into shared memory, beta, and one W_a_up row
+// per thread and unit.  t and W_b x must be final.
 template <int DK, int DV, class VS>
-__device__ void unit_gates(const FusedParams &P, VS *vs, int u, int slot, int vt, int t0, int nt)
-{
-    constexpr int hpu = 128 / DV;
-    const int b = u % P.Bs, kb = u / P.Bs, h0 = kb * hpu;
-    const int me = vt - t0;
-    if (me < 0 || me >= nt) return;
-    if (me < hpu) vs->beta[slot][me] = inv_one_plus_exp(-__ldcg(P.bpre + (size_t)b * P.nh + h0 + me));
-    const float *t = P.t + (size_t)b * P.r;
-    for (int i = me; i < hpu * DK; i += nt) {
-        const uint16_t *wr = P.wa_up + ((size_t)h0 * DK + i) * P.r;
-        float z = 0.f;
-        for (int j0 = 0; j0 < P.r; j0 += 32) {
-            uint4 w4[4];
-            float4 t4[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                w4[q] = j0 + q * 8 < P.r ? __ldg(reinterpret_cast<const uint4 *>(wr + j0 + q * 8)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                t4[q] = j0 + q * 4 < P.r ? __ldcg(reinterpret_cast<const float4 *>(t + j0 + q * 4)) : make_float4(0, 0, 0, 0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t wv[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
-                const float tv[8] = {t4[2 * q].x, t4[2 * q].y, t4[2 * q].z, t4[2 * q].w,
-                                     t4[2 * q + 1].x, t4[2 * q + 1].y, t4[2 * q + 1].z, t4[2 * q + 1].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    z = fmaf(bf16_bits_to_float(wv[e] & 0xFFFFu), tv[2 * e], z);
-                    z = fmaf(bf16_bits_to_float(wv[e] >> 16), tv[2 * e + 1], z);
-                }
-            }
-        }
-        vs->a[slot][i] = inv_one_plus_exp(z);
-    }
-}
-
-// Gates of this CTA's first two units (u1 < 0: none) into slots 0 and 1, by all 256 vector
-// threads with every load issued in one batch: t of the two sequences into shared memory,
-// beta, and one W_a_up row per thread and unit.  t and W_b x must be final.
-template <int DK, int DV, class VS>
-__device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt)
+__device__ void pair_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt)
 {
     constexpr int hpu = 128 / DV, rows = hpu * DK;
     const int r4 = P.r / 4;
@@ -556,7 +520,7 @@ __device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt
         const int j = (vt - 128) / hpu, hh = (vt - 128) % hpu;
         if (us[j] >= 0) {
             const int b = us[j] % P.Bs, h = (us[j] / P.Bs) * hpu + hh;
-            vs->beta[j][hh] = inv_one_plus_exp(-__ldcg(P.bpre + (size_t)b * P.nh + h));
+            P.gbuf[(size_t)us[j] * kGateStride + kGateBeta + hh] = inv_one_plus_exp(-__ldcg(P.bpre + (size_t)b * P.nh + h));
         }
     }
     for (int idx0 = 0; idx0 < 2 * rows; idx0 += 256) {
@@ -585,7 +549,7 @@ __device__ void first_gates(const FusedParams &P, VS *vs, int u0, int u1, int vt
                 }
             }
         }
-        if (has) vs->a[j][i] = inv_one_plus_exp(z);
+        if (has) P.gbuf[(size_t)us[j] * kGateStride + i] = inv_one_plus_exp(z);
     }
     named_bar(2, 256);
 }
@@ -652,11 +616,11 @@ __device__ void token_gates(const FusedParams &P, VS *vs, int bs, int kb, int vt
 
 // One state unit: sequence bs, o K-block kb (heads kb*128/dv ..), all dk rows, and its T
 // tokens applied in order (rows bs*T + t) with the state held in registers.  With one token
-// its gates are in slot nu & 1 and, while a few threads wait for the unit's q/k/v, the others
-// compute the gates of this CTA's next unit (next_u >= 0) into the other slot; with several
-// tokens every token's gates are computed here.
+// the first unit computes the gates of all of this CTA's units into the gate buffer (once
+// every CTA's gate rows are final) and each unit copies its own into slot nu & 1 while it
+// waits for its q/k/v; with several tokens every token's gates are computed here.
 template <int BP, int DK, int DV, bool MT, class VS>
-__device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, int next_u, int vt, int nu)
+__device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, int vt, int nu)
 {
     constexpr ActGeo G = act_geo(BP);
     const int T = MT ? P.T : 1, bs = u % P.Bs, kb = u / P.Bs, slot = nu & 1;
@@ -683,7 +647,14 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
         if (vt == 0 && !wait_count(P.ctr + C_GATE, P.t_gate, c, 10)) vs->fail = 1;
         named_bar(2, 256);
         if (vs->fail) return false;
-        if (!MT) first_gates<DK, DV>(P, vs, u, next_u, vt);
+        if (!MT)
+            for (int u2 = u; u2 < P.Bs * P.nKBo; u2 += 2 * (int)gridDim.x)
+                pair_gates<DK, DV>(P, vs, u2, u2 + (int)gridDim.x < P.Bs * P.nKBo ? u2 + (int)gridDim.x : -1, vt);
+    }
+    float ga = 0.f, gb = 0.f;  // this unit's gates (written by this CTA, read through L2)
+    if (!MT) {
+        if (vt < hpu * DK) ga = __ldcg(P.gbuf + (size_t)u * kGateStride + vt);
+        if (vt < hpu) gb = __ldcg(P.gbuf + (size_t)u * kGateStride + kGateBeta + vt);
     }
     // then the heads' q, k, v: wait for every segment of their row groups (one thread per
     // counter, so the round trips overlap), add the partials
@@ -695,11 +666,14 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
                                     : (vt < 2 * nq ? P.nRGq + glo + (vt - nq) : 2 * P.nRGq + vlo + (vt - 2 * nq));
             if (!wait_rb(P, key, c, 11)) vs->fail = 1;
         }
-        if (!MT && next_u >= 0 && nu >= 1) unit_gates<DK, DV>(P, vs, next_u, slot ^ 1, vt, 32, 224);
     }
     named_bar(2, 256);
     if (vt == 0 && nu < 2) KDA_TR(P, TR_USUB + 16 * nu + 1);
     if (vs->fail) return false;
+    if (!MT) {  // read after the items' barrier below
+        if (vt < hpu * DK) vs->a[slot][vt] = ga;
+        if (vt < hpu) vs->beta[slot][vt] = gb;
+    }
     if (MT) {
         token_gates<DK, DV>(P, vs, bs, kb, vt);
 #pragma unroll
@@ -906,7 +880,7 @@ __device__ void vector_role(const FusedParams &P, VS *vs, const Ctl &c)
         if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu);
         const int next = u + (int)gridDim.x < units ? u + (int)gridDim.x : -1;
         if (vt == 0 && next >= 0) prefetch_unit_state(P, next);  // its state streams in meanwhile
-        if (!state_unit<BP, DK, DV, MT>(P, vs, c, u, next, vt, nu)) return;
+        if (!state_unit<BP, DK, DV, MT>(P, vs, c, u, vt, nu)) return;
         if (vt == 0 && nu < 2) KDA_TR(P, TR_UNIT0 + 3 * nu + 2);
     }
     // out = sum of the W_o partials (both plane pairs): items of 32 output rows.  With tensor
@@ -1600,6 +1574,7 @@ size_t fused_scratch_bytes(const Dims &dmax, int num_sms)
     size_t n = 0;
     n += align_up((size_t)act_rows(g.gx, g.sr) * dmax.H, 1024);     // x planes + scale rows
     n += align_up((size_t)act_rows(g.go, g.sr) * dmax.Dv(), 1024);  // o planes + scale rows
+    n += align_up((size_t)std::min(dmax.B, kMaxBP) * (dmax.Dv() / 128) * kGateStride * 4, 256);  // gate buffer
     n += align_up(part, 256);                                // partial sums
     n += align_up(ctr_words(dmax, keys) * 4, 256);           // counters
     n += sched;                                              // tile lists, offsets, row-group info
@@ -1634,6 +1609,7 @@ void fused_bind_scratch(const Dims &dmax, int num_sms, void *base, size_t bytes,
     auto take = [&](size_t n, size_t a) { char *r = p; p += align_up(n, a); return r; };
     fs->xq = (uint8_t *)take((size_t)act_rows(g.gx, g.sr) * dmax.H, 1024);
     fs->oq = (uint8_t *)take((size_t)act_rows(g.go, g.sr) * dmax.Dv(), 1024);
+    fs->gbuf = (float *)take((size_t)std::min(dmax.B, kMaxBP) * (dmax.Dv() / 128) * kGateStride * 4, 256);
     fs->part = (float *)take(part, 256);
     fs->ctr_bytes = ctr_words(dmax, keys) * 4;
     fs->ctr = (uint32_t *)take(fs->ctr_bytes, 256);
@@ -1763,6 +1739,7 @@ cudaError_t fused_step(const Dims &d, int tokens, const kda_weights &w, const vo
     P.xq = fs.xq;
     P.oq = fs.oq;
     P.part = fs.part;
+    P.gbuf = fs.gbuf;
     P.q = s.q;
     P.k = s.k;
     P.v = s.v;

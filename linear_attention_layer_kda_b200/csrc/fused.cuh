@@ -80,6 +80,7 @@ struct FusedState {
     uint8_t *xq = nullptr;       // x planes  [act_rows(gx) rows][H]: E4M3 codes and fp32 block scales
     uint8_t *oq = nullptr;       // o planes  [act_rows(go) rows][Dv]
     float *part = nullptr;       // partial sums [nseg_total][2][BPmax][256]
+    float *gbuf = nullptr;       // gates of every single-token state unit [units][260]
     uint32_t *ctr = nullptr;     // flags and counters
     size_t ctr_bytes = 0;
     // one schedule per padded-batch class (BP 8, 16, 32, 64 up to the handle's largest)
