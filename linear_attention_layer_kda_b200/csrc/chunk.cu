@@ -1,8 +1,9 @@
 // chunk.cu -- the chunked (parallel-in-time) form of the gated delta rule, for prefill.
 //
-// The state S (dk x dv, fp32) of a head is carried through the sequence's tokens C at a time.  Inside a chunk that starts from S0, with
-// gamma(t, i) = prod_{i < j <= t} alpha_j the decay from token i to token t (a diagonal over
-// key channels) and g_t = gamma(t, start), unrolling the recurrence over the chunk gives
+// The state S (dk x dv, fp32) of a head is carried through the sequence's tokens C at a time.
+// Inside a chunk that starts from S0, with gamma(t, i) = prod_{i < j <= t} alpha_j the decay
+// from token i to token t (a diagonal over key channels) and g_t = gamma(t, start), unrolling
+// the recurrence over the chunk gives
 //
 //   u_t = beta_t (v_t - S0^T (g_t k^_t) - sum_{i < t} u_i k^_i^T gamma(t, i) k^_t)
 //   o_t = S0^T (g_t q_t) + sum_{i <= t} u_i k^_i^T gamma(t, i) q_t
