@@ -798,7 +798,6 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
                 *reinterpret_cast<uint32_t *>(P.oq + (size_t)o_row(p, row) * Dv + (size_t)kb * 128 + vc) = wq[p];
             if (lane == 0)
                 *reinterpret_cast<float *>(P.oq + (size_t)(G.rso + row / 32) * Dv + (size_t)kb * 128 + (row % 32) * 4) = sc;
-            fence_proxy_async_global();
             if (lane == 0 && nu < 2 && t == 0) KDA_TR(P, TR_USUB + 16 * nu + 6);
         }
         // S' = S~ + k^ u^T (kept in registers for the next token)
@@ -817,6 +816,7 @@ __device__ bool state_unit(const FusedParams &P, VS *vs, const Ctl &c, int u, in
         if (t + 1 < T) named_bar(2, 256);  // u, o and the reductions are reused by the next token
     }
     if (vw == 0) {
+        fence_proxy_async_global();  // every token's planes, read by other SMs' TMA copies
         __syncwarp();
         if (lane == 0) {
             // hand the release of the o block (every token's planes) to the o publisher (its
