@@ -268,7 +268,9 @@ KDA_API int kda_decode_set_launch_overlap(kda_handle h, int on);
  *   access).  Steps return KDA_ERR_INVALID_ARG until every peer is mapped.
  * After configuration every step of the handle (kda_decode_step, kda_decode_step_tokens)
  *   returns the whole out, and must take the fused engine (KDA_ERR_UNSUPPORTED_SHAPE, with
- *   nothing enqueued, for a batch it does not cover).  All ranks must issue the same steps
+ *   nothing enqueued, for a batch it does not cover).  kda_prefill is not a step of the
+ *   group: on a configured handle it still returns this rank's partial out (its heads' share),
+ *   which the caller sums over the ranks (a prompt's out is large and leaves the kernel anyway).  All ranks must issue the same steps
  *   in the same order: a step's kernel waits (bounded by the handle's timeout) for the
  *   matching step of every peer.  A timed-out wait leaves the group out of step; destroy
  *   and recreate the handles of every rank.  The regions are freed (peers unmapped) by

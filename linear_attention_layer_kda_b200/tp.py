@@ -132,6 +132,14 @@ class TensorParallelDecoder:
         if self.reduce == "nccl":
             self._dist.all_reduce(out, op=self._dist.ReduceOp.SUM, group=self.group)
 
+    def prefill(self, x, weights, state_shard, out, batch: int, tokens: int, chunk: int = 0) -> None:
+        """A prompt through the chunked form on this rank's heads; out ([batch * tokens, H], fp32)
+        becomes the whole layer's output on every rank (the partial outs summed with
+        torch.distributed.all_reduce in either mode: the prefill kernels do not exchange)."""
+        self.dec.prefill(x, weights, state_shard, out, batch, tokens, chunk)
+        if self._dist.is_initialized() and self._dist.get_world_size(self.group) > 1:
+            self._dist.all_reduce(out, op=self._dist.ReduceOp.SUM, group=self.group)
+
     def sync(self) -> None:
         self.dec.sync()
 

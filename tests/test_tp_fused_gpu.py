@@ -123,3 +123,28 @@ def test_configuration_errors_enqueue_nothing():
         assert torch.equal(st, tensors.state_tensor(inp.state0))
     finally:
         dec.close()
+
+
+def test_prefill_on_a_configured_handle():
+    """kda_prefill on a tensor-parallel handle returns the rank's partial out: with one rank,
+    the plain prefill's bits."""
+    import torch
+    from linear_attention_layer_kda_b200 import tensors, tp
+    shape = I.CONFIGS[1].replace(steps=48)
+    inp, w, _ = _setup(shape)
+    B, H, T = shape.batch, shape.hidden, 48
+    xs = tensors.bf16_tensor(np.stack([inp.x[t] for t in range(T)], axis=1).reshape(B * T, H))
+    plain = _decoder(shape)
+    group = tp.TensorParallelDecoder(inp, B)
+    try:
+        s1, s2 = tensors.state_tensor(inp.state0), tensors.state_tensor(inp.state0)
+        o1 = torch.empty(B * T, H, device="cuda")
+        o2 = torch.full((B * T, H), float("nan"), device="cuda")
+        plain.prefill(xs, w, s1, o1, B, T, 16)
+        group.prefill(xs, w, s2, o2, B, T, 16)
+        plain.sync()
+        group.sync()
+        assert torch.equal(o1, o2) and torch.equal(s1, s2)
+    finally:
+        group.close()
+        plain.close()
