@@ -41,6 +41,18 @@ def test_ragged_dk_ne_dv(engine):
     _assert_ok(errs, "ragged")
 
 
+# dk < dv: 64 key channels, 128 value columns per head (the remaining head shape)
+WIDE_V = I.KdaShape("wide_v_b3_h256_2x64x128", batch=3, hidden=256, num_heads=2, head_dk=64, head_dv=128,
+                    alpha_rank=32, steps=4, seed=23)
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+def test_dk_lt_dv(engine):
+    inp = I.generate(WIDE_V)
+    errs, _ = run_parity(inp, WIDE_V.steps, engine=engine)
+    _assert_ok(errs, "wide_v")
+
+
 @pytest.mark.parametrize("cfg", [1, 2])
 @pytest.mark.parametrize("engine", ENGINES)
 def test_full_size_single_step(cfg, engine):

@@ -59,8 +59,10 @@ def _check(got_out, got_state, ref_out, ref_state, T):
     assert es <= STATE_TOL, f"state error {es:.3e}"
 
 
+WIDE_V = I.KdaShape("wide_v_b3_h256_2x64x128", batch=3, hidden=256, num_heads=2, head_dk=64, head_dv=128,
+                    alpha_rank=32, steps=1, seed=53)
 CASES = [(I.CONFIGS[0], 64, 16), (I.CONFIGS[0], 64, 64), (I.CONFIGS[0], 4096, 64), (I.CONFIGS[0], 1000, 32),
-         (RAGGED, 100, 32), (RAGGED, 77, 16), (FULL, 256, 32), (FULL, 2048, 64)]
+         (RAGGED, 100, 32), (RAGGED, 77, 16), (WIDE_V, 90, 16), (WIDE_V, 90, 64), (FULL, 256, 32), (FULL, 2048, 64)]
 
 
 @pytest.mark.parametrize("shape,T,chunk", CASES, ids=[f"{s.name}_T{t}_C{c}" for s, t, c in CASES])
