@@ -19,9 +19,12 @@ namespace kda {
 SchedGeo fused_sched_geo(const Dims &dmax, int BP)
 {
     const ActGeo g = act_geo(BP);
-    const int nkb = dmax.H / 128;
-    const int run = BP <= 8 ? 2 : (BP <= 16 ? 4 : (BP <= 32 ? 8 : BP / 2));
-    return SchedGeo{g.nx, g.no, std::max(1, std::min(nkb, run))};
+    const int nkb = std::max(1, dmax.H / 128);
+    // longest run per padded batch (measured), then the K blocks of a row group cut into the
+    // fewest runs of equal length that respect it (48 blocks at 64 rows: 2 x 24, not 32 + 16)
+    const int longest = BP <= 8 ? 2 : (BP <= 16 ? 4 : (BP <= 32 ? 8 : BP / 2));
+    const int nrun = (nkb + longest - 1) / longest;
+    return SchedGeo{g.nx, g.no, (nkb + nrun - 1) / nrun};
 }
 
 // Tile order and segments.

@@ -65,6 +65,14 @@ def test_sched_geo(lib, BP, want):
     assert sched_geo(lib, BP, 4096, 32, 128, 128, 64) == want
 
 
+@pytest.mark.parametrize("BP,H,run", [(64, 6144, 24), (32, 6144, 8), (8, 6144, 2), (64, 384, 3), (8, 384, 2),
+                                      (16, 128, 1), (64, 5120, 20), (32, 1280, 5)])
+def test_runs_cut_the_k_blocks_evenly(lib, BP, H, run):
+    """A row group's K blocks are cut into the fewest equal runs no longer than the padded
+    batch's longest run (2, 4, 8, BP / 2)."""
+    assert sched_geo(lib, BP, H, H // 128, 128, 128, 64)[2] == run
+
+
 @pytest.mark.parametrize("P", [148, 132, 7])
 @pytest.mark.parametrize("H,nh,dk,dv,r", SHAPES)
 @pytest.mark.parametrize("BP", [8, 32, 64])
