@@ -14,8 +14,9 @@ namespace kda {
 // 32 and 64 sequences).  Runs: short ones spread each row group over more SMs, so its last
 // partial sum lands sooner, but every run writes a partial sum (BP x N fp32) and adds one to
 // the consumers' reads.  Measured at hidden 4096 (32 heads of 128 x 128): 2 tiles for 8
-// sequences (31.9 us against 32.5 us with 4), 4 for 16 (41.6 us against 48.7 us with 8),
-// BP / 2 for 64 (250.7 us; 252.5 us with 4); 8 for 32 sequences lies between.
+// sequences (31.9 us against 32.5 us with 4), 4 for 16 (41.6 us against 48.7 us with 8); 8 for
+// 32 sequences lies between.  At 64 sequences and hidden 6144 (48 K blocks): two runs of 24
+// (209 us) against 32 + 16 (233 us), 12 (220 us), 8 (235 us) or 48 (247 us).
 SchedGeo fused_sched_geo(const Dims &dmax, int BP)
 {
     const ActGeo g = act_geo(BP);
