@@ -43,7 +43,9 @@
  *     handle is unusable: every later call on it returns
  *     KDA_ERR_DEVICE_TIMEOUT; destroy it and create a new one.
  *   - The handle belongs to the device that was current at kda_decode_init;
- *     that device must be current whenever the handle enqueues work.
+ *     that device must be current whenever the handle enqueues work (a call
+ *     that would enqueue work on another current device returns
+ *     KDA_ERR_INVALID_ARG and enqueues nothing).
  *   - There is no CPU fallback: without a usable sm_100 device every call
  *     fails with KDA_ERR_NO_DEVICE or KDA_ERR_CUDA.
  *   - A handle is not thread-safe; use one handle per stream.

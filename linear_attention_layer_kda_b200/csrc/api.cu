@@ -30,6 +30,7 @@ struct kda_handle_s {
     cudaStream_t cstream = nullptr, ostream = nullptr;
     cudaEvent_t ev_x[2] = {}, ev_k[2] = {}, ev_o[2] = {};
     int hslot = 0;
+    bool host_async_ready = false;
     kda::FusedState fused;
     void *pf_ws = nullptr;   // prefill workspace (activations of every row), grown on demand
     kda::LtGemm *lt = nullptr;  // the prefill's GEMM library handle, created on first use
@@ -166,11 +167,30 @@ int take_device_status(kda_handle h)
     return fail(h, st, msg);
 }
 
+// Work is enqueued on the current device: it must be the handle's.
+int check_device(kda_handle h)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(h, KDA_ERR_NO_DEVICE, "no current CUDA device");
+    }
+    if (dev != h->device) return fail(h, KDA_ERR_INVALID_ARG, "the handle's device is not the current device");
+    return KDA_OK;
+}
+
 // A handle whose kernel could not drain its own copies after an abort is never used again.
-int check_usable(kda_handle h)
+int check_fatal(kda_handle h)
 {
     if (!h->fatal) return KDA_OK;
     return fail(h, KDA_ERR_DEVICE_TIMEOUT, "handle unusable: an aborted step did not drain its copies in flight");
+}
+
+// Before enqueueing work: the handle is usable and its device is current.
+int check_usable(kda_handle h)
+{
+    if (int rc = check_fatal(h)) return rc;
+    return check_device(h);
 }
 
 // A tensor-parallel handle runs only fused steps, and only once every peer is mapped.
@@ -430,6 +450,7 @@ int kda_tp_configure(kda_handle h, int rank, int world, void *ipc_handle_out)
     if (world < 1 || world > 8 || rank < 0 || rank >= world)
         return fail(h, KDA_ERR_INVALID_ARG, "need 1 <= world <= 8 and 0 <= rank < world");
     if (fs.tp_world) return fail(h, KDA_ERR_INVALID_ARG, "tensor parallelism is already configured");
+    if (int rc = check_device(h)) return rc;
     if (!fs.bytes) return fail(h, KDA_ERR_UNSUPPORTED_SHAPE, "the in-kernel reduction needs the fused engine");
     const size_t H = (size_t)h->cfg.hidden, bmax = (size_t)h->cfg.max_batch;
     fs.tp_slot_bytes = 2 * world * bmax * H * 4;
@@ -460,6 +481,7 @@ int kda_tp_set_peer(kda_handle h, int peer, const void *ipc_handle)
     if (!fs.tp_world) return fail(h, KDA_ERR_INVALID_ARG, "tensor parallelism is not configured");
     if (peer < 0 || peer >= fs.tp_world || peer == fs.tp_rank) return fail(h, KDA_ERR_INVALID_ARG, "bad peer rank");
     if (fs.tp_region[peer]) return fail(h, KDA_ERR_INVALID_ARG, "peer already mapped");
+    if (int rc = check_device(h)) return rc;
     cudaIpcMemHandle_t ipc;
     memcpy(&ipc, ipc_handle, sizeof ipc);
     void *p = nullptr;
@@ -536,18 +558,19 @@ int kda_decode_step_host(kda_handle h, const void *x_host, const kda_weights *w,
 
 static int host_async_setup(kda_handle h)
 {
-    if (h->ostream) return KDA_OK;
+    if (h->host_async_ready) return KDA_OK;
+    // each resource is created once: a call after a failed set-up creates only what is missing
     const size_t B = (size_t)h->cfg.max_batch, H = (size_t)h->cfg.hidden;
     cudaError_t e = cudaSuccess;
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
-        e = cudaMalloc(&h->hx[i], B * H * 2);
-        if (e == cudaSuccess) e = cudaMalloc(&h->hout[i], B * H * 4);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_x[i], cudaEventDisableTiming);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_k[i], cudaEventDisableTiming);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_o[i], cudaEventDisableTiming);
+        if (!h->hx[i]) e = cudaMalloc(&h->hx[i], B * H * 2);
+        if (e == cudaSuccess && !h->hout[i]) e = cudaMalloc(&h->hout[i], B * H * 4);
+        if (e == cudaSuccess && !h->ev_x[i]) e = cudaEventCreateWithFlags(&h->ev_x[i], cudaEventDisableTiming);
+        if (e == cudaSuccess && !h->ev_k[i]) e = cudaEventCreateWithFlags(&h->ev_k[i], cudaEventDisableTiming);
+        if (e == cudaSuccess && !h->ev_o[i]) e = cudaEventCreateWithFlags(&h->ev_o[i], cudaEventDisableTiming);
     }
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cstream, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->ostream, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !h->cstream) e = cudaStreamCreateWithFlags(&h->cstream, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !h->ostream) e = cudaStreamCreateWithFlags(&h->ostream, cudaStreamNonBlocking);
     // the slots start free: their "step done" and "out copied" events complete at once
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
         e = cudaEventRecord(h->ev_k[i], h->cstream);
@@ -557,6 +580,7 @@ static int host_async_setup(kda_handle h)
         (void)cudaGetLastError();
         return fail(h, KDA_ERR_OUT_OF_MEMORY, "host-step staging allocation failed");
     }
+    h->host_async_ready = true;
     return KDA_OK;
 }
 
@@ -698,6 +722,7 @@ static int state_copy(kda_handle h, void *dst, const void *src, int seq0, int ns
     if (!dst || !src) return fail(h, KDA_ERR_INVALID_ARG, "null state or host buffer");
     if (seq0 < 0 || nseq < 1 || (long long)seq0 + nseq > h->cfg.max_batch)
         return fail(h, KDA_ERR_INVALID_ARG, "need seq0 >= 0, nseq >= 1 and seq0 + nseq <= max_batch");
+    if (int rc = check_device(h)) return rc;
     const kda_config &c = h->cfg;
     const size_t per_seq = (size_t)c.num_heads * c.head_dk * c.head_dv * 4;
     const size_t off = (size_t)seq0 * per_seq, n = (size_t)nseq * per_seq;
@@ -726,7 +751,7 @@ int kda_decode_sync(kda_handle h)
     if (e == cudaSuccess && h->ostream) e = cudaStreamSynchronize(h->ostream);
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
     const int st = take_device_status(h);
-    return st ? st : check_usable(h);
+    return st ? st : check_fatal(h);
 }
 
 int kda_decode_debug_copy(kda_handle h, int which, void *dst, size_t bytes)
