@@ -148,3 +148,41 @@ def test_prefill_on_a_configured_handle():
     finally:
         group.close()
         plain.close()
+
+
+def test_nccl_reduce_mode_at_one_rank(tmp_path):
+    """reduce="nccl": the local step, then torch.distributed.all_reduce of out over NCCL.  With
+    one rank the sum is the rank's own out, so it must equal the plain step bit for bit."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from linear_attention_layer_kda_b200 import tensors, tp
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised in this process")
+    store = dist.FileStore(str(tmp_path / "store"), 1)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        shape = I.CONFIGS[1].replace(steps=3)
+        inp, w, _ = _setup(shape)
+        B, H = shape.batch, shape.hidden
+        plain = _decoder(shape)
+        group = tp.TensorParallelDecoder(inp, B, reduce="nccl")
+        try:
+            s1, s2 = tensors.state_tensor(inp.state0), tensors.state_tensor(inp.state0)
+            o1 = torch.empty(B, H, device="cuda")
+            o2 = torch.full((B, H), float("nan"), device="cuda")
+            for t in range(shape.steps):
+                x = tensors.bf16_tensor(inp.x[t])
+                plain.step(x, w, s1, o1)
+                group.step(x, w, s2, o2)
+                plain.sync()
+                group.sync()
+                torch.cuda.synchronize()
+                assert torch.equal(o1, o2), f"step {t}: out differs from the plain step"
+            assert torch.equal(s1, s2)
+        finally:
+            group.close()
+            plain.close()
+    finally:
+        dist.destroy_process_group()
