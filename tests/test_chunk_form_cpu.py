@@ -33,9 +33,16 @@ def chunk_step(S0, q, k, v, beta, alpha):
     return O, S
 
 
+SHAPES = [I.CONFIGS[0],  # batch 1, hidden 256, 2 heads of 64 x 64, 16 steps
+          I.KdaShape("chunk_dk_lt_dv", batch=1, hidden=256, num_heads=2, head_dk=64, head_dv=128,
+                     alpha_rank=32, steps=12, seed=31),
+          I.KdaShape("chunk_dk_gt_dv", batch=1, hidden=384, num_heads=2, head_dk=128, head_dv=64,
+                     alpha_rank=32, steps=12, seed=32)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: s.name)
 @pytest.mark.parametrize("C", [1, 4, 5, 16])
-def test_chunked_form_matches_the_recurrence(C):
-    shape = I.CONFIGS[0]  # batch 1, hidden 256, 2 heads of 64 x 64, 16 steps
+def test_chunked_form_matches_the_recurrence(C, shape):
     T, nh, dk, dv = shape.steps, shape.num_heads, shape.head_dk, shape.head_dv
     inp = I.generate(shape)
     m = oracle.OracleModel(inp, batch=1)
